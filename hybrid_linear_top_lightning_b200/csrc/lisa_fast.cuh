@@ -1,0 +1,37 @@
+// Specialised sm_100a paths.  Each `*_supported` predicate says whether a call
+// can take the specialised kernel (shape, dtype and pointer alignment); the
+// API falls back to the generic kernels otherwise.
+#pragma once
+
+#include "lisa_internal.cuh"
+
+namespace lisa {
+
+// Fused decode step (decode_fused.cu).
+size_t fast_decode_ws_bytes(const Shape& s);
+bool fast_decode_supported(const Shape& s, const lisa_decode_args& a);
+cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st);
+
+// Top-M over many query rows (prefill).
+size_t fast_topm_ws_bytes(const Shape& s);
+bool fast_topm_supported(const Shape& s, const void* q_I, const void* k_I, const float* w,
+                         int64_t w_tok_stride);
+cudaError_t fast_topm(const Shape& s, const void* q_I, const void* k_I, const float* w,
+                      int64_t w_tok_stride, int32_t* idx, int32_t* count, void* ws,
+                      cudaStream_t st);
+
+// Sparse / dense attention.
+size_t fast_attention_ws_bytes(const Shape& s, bool dense);
+bool fast_attention_supported(const Shape& s, const void* q, const void* k, const void* v,
+                              bool dense);
+cudaError_t fast_attention(const Shape& s, const void* q, const void* k, const void* v,
+                           const int32_t* idx, const int32_t* count, void* o, void* ws,
+                           cudaStream_t st);
+
+// Chunked linear-attention prefill.
+size_t fast_linear_prefill_ws_bytes(const Shape& s);
+bool fast_linear_prefill_supported(const Shape& s, const void* q, const void* k, const void* v);
+cudaError_t fast_linear_prefill(const Shape& s, const void* q, const void* k, const void* v,
+                                float* S, float* z, void* o, void* ws, cudaStream_t st);
+
+}  // namespace lisa

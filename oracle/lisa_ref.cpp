@@ -121,8 +121,8 @@ void ref_index_scores(const RefDims* D, const float* q_I, const float* k_I,
 }
 
 // ---------------------------------------------------------------------------
-// Top-M selection (Sec. 3.2: "select the M positions with the largest values"
-// over the summed indexer scores; the paper calls it top-M (argmax)).  All
+// Top-M selection (Sec. 3.2, "Indexer-Guided Token Selection": the summed
+// indexer scores pick the M highest-scoring positions).  All
 // candidates s <= p are sorted by (score descending, position ascending); the
 // first min(M, p+1) are kept.  Output: the kept positions in ascending order,
 // padded with -1 to M entries; count = min(M, p+1).
@@ -183,8 +183,8 @@ static void attend(const RefDims* D, const float* qh, const float* k_cache,
 }
 
 // ---------------------------------------------------------------------------
-// Sparse self-attention SA_M over the selected positions (Sec. 3.2, Eq. 1 and
-// "we fill the cached ... at the corresponding positions into SA_M"): query
+// Sparse self-attention SA_M over the selected positions (Sec. 3.2, Eq. 1; the
+// cached entries at the chosen positions feed SA_M): query
 // head h attends with KV head g = h / (H_q / H_kv) over the count[b, r] valid
 // entries of idx[b, r, :].  q: [B, T, H_q, d]; caches: [B, N_max, H_kv, d];
 // idx: [B, R, M]; o: [B, R, H_q, d].
@@ -229,8 +229,8 @@ void ref_dense_attn(const RefDims* D, const float* q, const float* k_cache,
     }
 }
 
-// Feature map of the linear branch: identity (Sec. 3.1, "setting phi to the
-// identity function and removing the normalization term"), or elu(x) + 1.
+// Feature map of the linear branch: identity with no normaliser (the choice
+// Sec. 3.1 adopts), or elu(x) + 1.
 static inline double feature(int phi, double x) {
     if (phi == 0) return x;
     return x > 0.0 ? x + 1.0 : std::exp(x);
