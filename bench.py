@@ -1,0 +1,403 @@
+"""Benchmark of liblisa on B200: the LISA decode step of a 7B-shaped layer at 16K context.
+
+Workload (one "step" = one pass of the whole hot path over one batch): the
+fused decode step — cache append, linear-state update and read-out, indexer
+scan over the full context, top-M, sparse attention over the selected rows
+and the gate — for B=8 sequences at context 16384 (28 query / 4 KV heads,
+head dim 128, 8 indexer heads of dim 64, M=2048), bf16 activations, fp32
+linear state built by a prefill of the same seeded tokens.
+
+Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
+the launching stream; L2 is flushed (a 256 MB write) before every timed step
+and outside its events.  A barrier and a device synchronise bracket the timed
+region; the reported time is the maximum over ranks.  Under torchrun each rank
+runs its own replica of the workload (weak scaling; the path has no exchange).
+
+`--impl reference` times the CPU oracle (plain fp64 C++) on the host cores on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LISA decode tok/s @16K ctx (7B-shape layer), prefill tok/s, % of HBM roofline"
+UNIT = "tok/s"
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def decode_bytes(wl) -> dict:
+    """Algorithmic HBM bytes of one decode step (per sequence and total).
+
+    Keys are read once (k_I scan over the n cached positions), only the
+    min(M, n) selected K/V rows are gathered, the fp32 state is read and
+    written once, plus the step's small inputs and outputs."""
+    n, M = wl.n, wl.M
+    scan = n * wl.H_Ik * wl.d_I * 2
+    gather = min(M, n) * wl.H_kv * wl.d * 2 * 2
+    state = wl.H_kv * wl.d * wl.d * 4 * 2
+    small = (wl.H_q * wl.d * 2 * 2          # q, o
+             + wl.H_q * wl.d * 2            # q_L (aliases q, counted once more for the LA read)
+             + wl.H_kv * wl.d * 2 * 2 * 2   # k_new, v_new read + written to the cache
+             + wl.H_I * wl.d_I * 2          # q_I
+             + wl.d_I * wl.H_Ik * 2 * 2     # k_I_new read + written
+             + wl.H_I * 4 + wl.H_q * 2)     # w, gate logits
+    per_seq = scan + gather + state + small
+    return dict(scan=scan, gather=gather, state=state, small=small, per_seq=per_seq,
+                total=per_seq * wl.B)
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode_fused.cu", "sm100_ptx.cuh", "lisa_internal.cuh"):
+        with open(os.path.join(ROOT, "hybrid_linear_top_lightning_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(wl):
+    """DRAM bytes per launch of the fused decode kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "decode_fused_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_source_sha") != _kernel_source_hash():
+        return None
+    if rec.get("workload") != wl.name:
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def _setup_decode(wl, device):
+    import torch
+
+    from hybrid_linear_top_lightning_b200 import inputs, lisa
+
+    gen = inputs.Generator(wl)
+    n, p, B = wl.n, wl.n - 1, wl.B
+    bf = torch.bfloat16
+    kc = torch.empty(B, n, wl.H_kv, wl.d, dtype=bf, device=device)
+    vc = torch.empty_like(kc)
+    kIc = torch.empty(B, n, wl.H_Ik, wl.d_I, dtype=bf, device=device)
+    for b in range(B):
+        kc[b] = torch.from_numpy(gen.k(b, 0, n)).to(bf)
+        vc[b] = torch.from_numpy(gen.v(b, 0, n)).to(bf)
+        kIc[b] = torch.from_numpy(gen.k_I(b, 0, n)).to(bf)
+    host = {
+        "q": gen.batch("q", p, n), "q_I": gen.batch("q_I", p, n), "w": gen.batch("w", p, n),
+        "gate": gen.batch("gate", p, n),
+        "k_new": np.ascontiguousarray(kc[:, p:].float().cpu().numpy()),
+        "v_new": np.ascontiguousarray(vc[:, p:].float().cpu().numpy()),
+        "k_I_new": np.ascontiguousarray(kIc[:, p:].float().cpu().numpy()),
+    }
+    # linear state of the n-1 cached tokens, built by the library's own prefill
+    S = torch.zeros(B, wl.H_kv, wl.d, wl.d, dtype=torch.float32, device=device)
+    Dp = lisa.make_dims(B, p, 0, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                        chunk=wl.chunk)
+    ws_p = lisa.workspace(Dp, lisa.LISA_OP_LINEAR_PREFILL, device)
+    o_tmp = torch.empty(B, p, wl.H_q, wl.d, dtype=bf, device=device)
+    q_tmp = torch.zeros(B, p, wl.H_q, wl.d, dtype=bf, device=device)
+    lisa.lisa_linear_prefill(Dp, q_tmp, kc[:, :p].contiguous(), vc[:, :p].contiguous(), S, None,
+                             o_tmp, ws_p)
+    del o_tmp, q_tmp, ws_p
+    dev = {k: torch.from_numpy(v).to(torch.float32 if k == "w" else bf).to(device)
+           for k, v in host.items()}
+    return kc, vc, kIc, S, dev, host
+
+
+def run_gpu(args, wl, rank, world, device):
+    import torch
+    import torch.distributed as dist
+
+    from hybrid_linear_top_lightning_b200 import lisa
+
+    torch.manual_seed(0)
+    kc, vc, kIc, S, dv, host = _setup_decode(wl, device)
+    B, n, p = wl.B, wl.n, wl.n - 1
+    D = lisa.make_dims(B, 1, p, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M)
+    ws = lisa.workspace(D, lisa.LISA_OP_DECODE_STEP, device)
+    o = torch.empty(B, 1, wl.H_q, wl.d, dtype=torch.bfloat16, device=device)
+    a = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"], dv["w"],
+                         wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"], kc, vc, kIc, S,
+                         None, o)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lisa.lisa_decode_step(D, a, ws, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    assert lisa.lisa_check_status(ws, stream) == lisa.LISA_OK
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        gpu_id = str(device.index)
+    with ClockSampler(gpu_id) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    assert lisa.lisa_check_status(ws, stream) == lisa.LISA_OK
+    total_ms = sum(times_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
+        torch.float32 if k == "w" else torch.bfloat16).pin_memory() for k, v in host.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in pinned.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for k, x in pinned.items():
+            dv[k].copy_(x, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        flush.fill_(1)
+        e2e_step()
+    torch.cuda.synchronize()
+    e_st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_st[i].record(stream)
+        e2e_step()
+        e_en[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_st, e_en))
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+
+    bytes_ = decode_bytes(wl)
+    avg_s = total_ms / 1e3 / args.steps
+    hbm_peak, _, peak_kind = _peaks()
+    achieved = bytes_["total"] / avg_s / 1e9
+    value = world * B * args.steps / (total_ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Philox inputs, 1% planted heavy keys)",
+        "config": {"workload": wl.name, "B": B, "context": n, "H_q": wl.H_q, "H_kv": wl.H_kv,
+                   "d": wl.d, "H_I": wl.H_I, "d_I": wl.d_I, "M": wl.M,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "step": "fused decode step: append, linear update+readout, indexer scan, "
+                           "top-M, sparse attention, gate"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "frac_of_8TBs": achieved / 8000.0,
+                     "traffic": _profiled_traffic(wl),
+                     "algorithmic_bytes_per_launch": bytes_["total"],
+                     "kernel": "k_decode_fused", "launch_us": avg_s * 1e6},
+        "e2e": {"value": world * B * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "step_ms_min": min(times_ms), "step_ms_median": statistics.median(times_ms),
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_decode_sample(wl, seqs: int, budget_s: float):
+    """Time the oracle's decode step on `seqs` sequences of the workload, repeated
+    until about `budget_s` seconds have passed.  Returns (tok/s, threads, note)."""
+    from hybrid_linear_top_lightning_b200 import inputs
+    from oracle import ref
+
+    gen = inputs.Generator(wl.with_(B=seqs))
+    n, p = wl.n, wl.n - 1
+    kc = gen.batch("k", 0, n)
+    vc = gen.batch("v", 0, n)
+    kI = gen.batch("k_I", 0, n)
+    q = gen.batch("q", p, n)
+    qI = gen.batch("q_I", p, n)
+    w = gen.batch("w", p, n)
+    gl = gen.batch("gate", p, n)
+    rng = np.random.default_rng(0)
+    S0 = rng.standard_normal((seqs, wl.H_kv, wl.d, wl.d)) * 0.1
+    D = ref.Dims(B=seqs, T=1, n_past=p, N_max=n, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d, H_I=wl.H_I,
+                 H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        ref.forward(D, q, kc, vc, qI, kI, w, wl.H_I, q, kc[:, p:], vc[:, p:], gl, S0=S0)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    tok_s = reps * seqs / el
+    return tok_s, ref.num_threads(), (f"{reps} oracle decode steps of {seqs} sequences at "
+                                      f"context {n} (full step per sequence) in {el:.1f} s")
+
+
+def run_reference(args, wl):
+    tok_s, cores, note = oracle_decode_sample(wl, seqs=wl.B, budget_s=max(5.0, args.cpu_seconds))
+    return {
+        "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": wl.B / tok_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "context": wl.n, "M": wl.M},
+        "impl": "reference",
+        "cpu_baseline": {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": note},
+        "e2e": {"value": tok_s, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from hybrid_linear_top_lightning_b200 import inputs
+
+    wl = inputs.DECODE_7B
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        line = run_gpu(args, wl, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            tok_s, cores, note = oracle_decode_sample(wl, seqs=2, budget_s=args.cpu_seconds)
+            line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores,
+                                    "kind": "oracle", "sample": note}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -18,10 +18,5 @@ bool fast_linear_prefill_supported(const Shape&, const void*, const void*, const
 cudaError_t fast_linear_prefill(const Shape&, const void*, const void*, const void*, float*, float*,
                                 void*, void*, cudaStream_t) { return cudaErrorNotSupported; }
 
-size_t fast_decode_ws_bytes(const Shape&) { return 0; }
-bool fast_decode_supported(const Shape&, const lisa_decode_args&) { return false; }
-cudaError_t fast_decode_step(const Shape&, const lisa_decode_args&, void*, cudaStream_t) {
-    return cudaErrorNotSupported;
-}
 
 }  // namespace lisa

@@ -204,10 +204,14 @@ def lisa_gate_fuse(dims, gate_logit_lin, o_lin, o_sparse, o, stream=None):
 
 def decode_args(q, k_new, v_new, q_I, k_I_new, w, w_tok_stride, q_L, k_L, v_L, gate_logit_lin,
                 k_cache, v_cache, k_I_cache, S, z, o, idx=None, count=None) -> lisa_decode_args:
-    return lisa_decode_args(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_I), _ptr(k_I_new), _ptr(w),
+    args = lisa_decode_args(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_I), _ptr(k_I_new), _ptr(w),
                             int(w_tok_stride), _ptr(q_L), _ptr(k_L), _ptr(v_L),
                             _ptr(gate_logit_lin), _ptr(k_cache), _ptr(v_cache), _ptr(k_I_cache),
                             _ptr(S), _ptr(z), _ptr(o), _ptr(idx), _ptr(count))
+    # the struct holds raw device pointers: keep the tensors alive with it
+    args._keep = (q, k_new, v_new, q_I, k_I_new, w, q_L, k_L, v_L, gate_logit_lin, k_cache,
+                  v_cache, k_I_cache, S, z, o, idx, count)
+    return args
 
 
 def lisa_decode_step(dims, args: lisa_decode_args, ws, stream=None):

@@ -121,7 +121,11 @@ def dense_attn(D: Dims, q, k_cache, v_cache, rows=None) -> np.ndarray:
 
 def linear(D: Dims, q_L, k_L, v_L, S0=None, z0=None, rows=None):
     """Returns (o [B,R,H_q,d], S [B,H_kv,d,d], z [B,H_kv,d] or None)."""
-    q_L, k_L, v_L = _f32(q_L), _f32(k_L), _f32(v_L)
+    if q_L is None:  # only allowed when no output row is requested
+        assert rows is not None and len(rows) == 0
+    else:
+        q_L = _f32(q_L)
+    k_L, v_L = _f32(k_L), _f32(v_L)
     r, R = _rows(D, rows)
     S = np.zeros((D.B, D.H_kv, D.d, D.d)) if S0 is None else np.array(S0, dtype=np.float64)
     z = None
