@@ -40,6 +40,7 @@ EXPORTS = (
     "lisa_index_scores", "lisa_topm", "lisa_sparse_attn", "lisa_linear_prefill",
     "lisa_linear_decode", "lisa_gate_fuse", "lisa_decode_step", "lisa_dense_attn",
     "lisa_workspace_size", "lisa_check_status", "lisa_status_string", "lisa_version",
+    "lisa_topm_noalloc",
 )
 
 
@@ -92,6 +93,7 @@ def load() -> ctypes.CDLL:
         "lisa_dense_attn": [dp, vp, vp, vp, vp, vp, sz, vp],
         "lisa_workspace_size": [dp, ctypes.c_int, ctypes.POINTER(sz)],
         "lisa_check_status": [vp, vp],
+        "lisa_topm_noalloc": [dp, vp, vp, vp, i64, vp, vp, vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -171,6 +173,13 @@ def lisa_topm(dims, q_I, k_I_cache, w, w_tok_stride, idx, count, ws, stream=None
     _check(load().lisa_topm(ctypes.byref(dims), _ptr(q_I), _ptr(k_I_cache), _ptr(w),
                             int(w_tok_stride), _ptr(idx), _ptr(count), _ptr(ws), ws.numel(),
                             _stream(stream)), "lisa_topm")
+
+
+def lisa_topm_noalloc(dims, q_I, k_I_cache, w, w_tok_stride, idx, count, stream=None):
+    """lisa_topm without a workspace (scores kept in the library's built-in 4 MiB array)."""
+    _check(load().lisa_topm_noalloc(ctypes.byref(dims), _ptr(q_I), _ptr(k_I_cache), _ptr(w),
+                                    int(w_tok_stride), _ptr(idx), _ptr(count), _stream(stream)),
+           "lisa_topm_noalloc")
 
 
 def lisa_sparse_attn(dims, q, k_cache, v_cache, idx, count, o_sparse, ws, stream=None):

@@ -193,6 +193,25 @@ LISA_API lisa_status lisa_dense_attn(const lisa_dims* dims, const void* q, const
                             const void* v_cache, void* o, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* lisa_topm without a workspace, for callers that cannot allocate device memory
+ * for the library (a host framework whose allocator is off-limits, plugin or
+ * callback interfaces that pass only the call's tensors, loops where a
+ * cudaMalloc and its device synchronisation are not acceptable).  The paper
+ * has no counterpart: this is a packaging variant of lisa_topm.  Same inputs,
+ * outputs and result as lisa_topm; the scores of the call are kept in a 4 MiB
+ * device array built into the library, held on every GPU that loads it until
+ * the process exits.
+ *  - Calls needing more than 4 MiB of scores (B*T*(n_past+T) floats) return
+ *    LISA_ERR_UNSUPPORTED without launching anything.
+ *  - The array is shared by every call on a device and keeps the last call's
+ *    contents; calls that may overlap on the GPU race on it, so the caller must
+ *    order them (one stream, or explicit events).
+ *  - The first call on each device sets up the array's device address (with
+ *    that device current); make that first call before any stream capture. */
+LISA_API lisa_status lisa_topm_noalloc(const lisa_dims* dims, const void* q_I, const void* k_I_cache,
+                              const float* w, int64_t w_tok_stride, int32_t* idx, int32_t* count,
+                              void* stream);
+
 /* Workspace bytes needed by `op` for these dims (0 if none). */
 LISA_API lisa_status lisa_workspace_size(const lisa_dims* dims, int op, size_t* bytes);
 

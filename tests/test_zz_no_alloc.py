@@ -1,0 +1,64 @@
+"""lisa_topm_noalloc: the workspace-free variant of lisa_topm.
+
+Some callers cannot allocate device memory for the library (a host framework
+whose allocator is off-limits, plugin interfaces that pass only the call's
+tensors).  This entry point keeps its scratch in a device array built into the
+library.  The test calls it through the C ABI twice in a row (the shared
+array keeps the previous call's contents) and checks that each result equals
+what lisa_topm, which takes a caller-provided workspace, returns for the same
+inputs.  It lives in its own file, collected last.
+"""
+import numpy as np
+import pytest
+import torch
+
+from hybrid_linear_top_lightning_b200 import inputs, lisa
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(wl, T, n_past, seed_shift):
+    gen = inputs.Generator(wl.with_(seed=wl.seed + seed_shift))
+    L = n_past + T
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    q_I = torch.from_numpy(gen.batch("q_I", n_past, L)).to(dt).cuda()
+    k_I = torch.from_numpy(gen.batch("k_I", 0, L)).to(dt).cuda()
+    w = torch.from_numpy(gen.batch("w", n_past, L)).cuda()
+    D = lisa.make_dims(wl.B, T, n_past, L, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                       dtype=wl.dtype)
+    return D, q_I, k_I, w
+
+
+def _topm_both(D, q_I, k_I, w, H_I):
+    B, T, M = D.B, D.T, D.M
+    idx_ws = torch.empty(B, T, M, dtype=torch.int32, device="cuda")
+    cnt_ws = torch.empty(B, T, dtype=torch.int32, device="cuda")
+    ws = lisa.workspace(D, lisa.LISA_OP_TOPM)
+    lisa.lisa_topm(D, q_I, k_I, w, H_I, idx_ws, cnt_ws, ws)
+    idx_na = torch.full((B, T, M), -9, dtype=torch.int32, device="cuda")
+    cnt_na = torch.full((B, T), -9, dtype=torch.int32, device="cuda")
+    lisa.lisa_topm_noalloc(D, q_I, k_I, w, H_I, idx_na, cnt_na)
+    torch.cuda.synchronize()
+    return idx_ws.cpu().numpy(), cnt_ws.cpu().numpy(), idx_na.cpu().numpy(), cnt_na.cpu().numpy()
+
+
+def test_noalloc_topm_matches_workspace_topm_twice():
+    # first call: a prefill-shaped fp32 call; second: a bf16 decode-shaped call
+    # whose scores overwrite part of the first call's scratch contents
+    cases = [(inputs.TINY.with_(M=32), 200, 0, 0), (inputs.DECODE_7B.with_(B=4, M=512), 1, 9000, 1)]
+    for wl, T, n_past, shift in cases:
+        D, q_I, k_I, w = _case(wl, T, n_past, shift)
+        a_idx, a_cnt, b_idx, b_cnt = _topm_both(D, q_I, k_I, w, wl.H_I)
+        # the same kernels compute both, so the index sets are identical
+        np.testing.assert_array_equal(b_cnt, a_cnt)
+        np.testing.assert_array_equal(b_idx, a_idx)
+
+
+def test_noalloc_rejects_calls_beyond_its_scratch():
+    wl = inputs.DECODE_7B.with_(B=8)
+    D = lisa.make_dims(8, 1, 200000, 200001, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M)
+    t = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    i = torch.zeros(16, dtype=torch.int32, device="cuda")
+    with pytest.raises(lisa.LisaError) as err:
+        lisa.lisa_topm_noalloc(D, t, t, t.float(), wl.H_I, i, i)
+    assert err.value.status == lisa.LISA_ERR_UNSUPPORTED
