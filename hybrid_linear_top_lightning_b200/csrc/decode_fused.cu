@@ -1,40 +1,42 @@
-// Fused LISA decode step for B200 (sm_100a): one kernel launch per step.
+// LISA decode step for B200 (sm_100a): three kernels chained by programmatic
+// dependent launch (each starts launching while its predecessor runs), every
+// SM busy, no inter-CTA waiting.
 //
-// One thread-block cluster of C CTAs serves one sequence.  CTA r of the
-// cluster owns the key slice [r*KPC, (r+1)*KPC) of the context and the slice
-// of linear-state columns that its (KV head, column block) names.  The step
-// (LISA, arXiv 2607.19358v1: Sec. 3.2 generation step and Eq. 1; Sec. 3.1 and
-// Sec. 3.3 Eq. 3-4 for the linear branch):
+// Step semantics (LISA, arXiv 2607.19358v1: the generation step of Sec. 3.2 and
+// Eq. 1; Sec. 3.1 and Sec. 3.3 Eq. 3-4 for the linear branch): append the new
+// token, score every cached key with the Lightning Indexer, keep the top M,
+// attend over them, run the linear branch, mix the two with the gate.
 //
-//  A  indexer scan: the CTA's k_I rows stream in by TMA (128-row boxes,
-//     128-byte swizzle, a ring of stages); each warp scores 16 keys at a time
-//     on the tensor cores (mma m16n8k16: keys x indexer heads, K = d_I = 64),
-//     then ReLU, head weights and the head sum give the score, kept in shared
-//     memory.  The new token's row comes from k_I_new.  Meanwhile the CTA's
-//     linear-state slice arrives by cp.async.
-//  A' linear branch: S[:, cols] += phi(k)^T v[cols]; o_lin = phi(q) S[:, cols]
-//     (divided by phi(q).z in elu+1 mode) for the query heads of the group.
-//  B  top-M: an exact radix select over the cluster (11/11/10-bit passes on the
-//     order-preserving integer key of each score).  Each CTA histograms its own
-//     keys and adds the non-zero bins into the bin owner's shared memory
-//     (distributed shared memory); after a cluster barrier every CTA reads the
-//     whole histogram and finds the same digit.  Ties at the threshold keep the
-//     lowest positions.  The selected positions are then spread evenly over
-//     the CTAs (each CTA writes its picks straight into the owner's list).
-//  C  sparse attention: each CTA gathers its share of the selected K and V rows
-//     (all KV heads of a position are one contiguous row) with 1D bulk copies
-//     into padded shared-memory rows, and runs an online softmax on the tensor
-//     cores: query heads of a group on the M side (16 rows), keys on N.
-//  D  combine: per-CTA partial (max, sum, output) triples are merged across the
-//     cluster through distributed shared memory; the gate mixes the linear and
-//     sparse outputs and writes o.
+// K1 scan (grid B x S1, 8 scan warps + 4 linear-branch warps per CTA).
+//    Scan warps: CTA j of sequence b scores keys [j*KPC, (j+1)*KPC).  The k_I
+//    rows arrive by TMA (128-row boxes, 128-byte swizzle, eight in flight); a
+//    warp scores 16 keys at a time on the tensor cores (mma m16n8k16: keys x
+//    indexer heads, K = d_I), then ReLU, head weights and head sum.  Scores go
+//    to a workspace row; each slice also adds its histogram of the top 12 bits
+//    of the order-preserving score keys into the sequence's histogram.
+//    Linear-branch warps (concurrently): one slice (sequence, KV head, 32
+//    value columns) of S += phi(k)^T v and o_lin = phi(q) S (/ phi(q).z).
+//    CTA 0 of each sequence appends the new k, v, k_I to the caches.
+// K2 attend (grid B x S2, 256 threads).  Each CTA derives the exact top-M set
+//    by itself: the first 12-bit digit from the histogram, then one ordered
+//    pass over the score row (TMA-loaded into shared memory) collecting the
+//    keys of that digit, two 10-bit refinements over those candidates only,
+//    and a ranked walk (warp ballots and scans) that extracts this CTA's even
+//    share of the selected positions.  Ties keep the lowest positions.  The
+//    share's K and V rows (all KV heads of a position are one row) are
+//    gathered with 128-bit loads through registers into padded shared-memory
+//    rows and attended with an online softmax on the tensor cores.  Partial
+//    (max, sum, output) triples go to the workspace.
+// K3 combine (grid B x H_q, one thread per output dim): merges the partials,
+//    gates with the linear branch, writes o; advances z (elu+1 mode) and clears
+//    the histogram for the next call.
 //
-// Every wait on an mbarrier is bounded; a wait that gives up records
-// LISA_ERR_TIMEOUT in the status word, skips the dependent work and still
-// takes part in every cluster barrier, so no CTA is left waiting.  There are no
-// inter-cluster dependencies and no spin loops on global memory.
+// The only waits are on TMA mbarriers, each bounded: a wait that gives up
+// records LISA_ERR_TIMEOUT in the status word and dependent work is skipped.
 #include <cuda.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
@@ -45,26 +47,28 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kD = 128;             // head dimension of this path
-constexpr int kDI = 64;             // indexer dimension of this path
-constexpr int kScanRows = 128;      // keys per TMA box (16 per warp)
-constexpr int kScanStages = 4;      // TMA ring depth (64 KB in flight)
-constexpr int kScanBoxBytes = kScanRows * kDI * 2;
-constexpr int kGKeys = 32;          // keys per gather stage
-constexpr int kGStages = 2;
-constexpr int kMaxKPC = 8192;       // keys per CTA (scores kept in shared memory)
-constexpr int kMaxPer = 512;        // selected positions per CTA after balancing
-constexpr int kMaxBins = 2048;
-constexpr uint32_t kWaitTries = 1u << 22;  // bounded mbarrier polls
+constexpr int kD = 128;               // head dimension of this path
+constexpr int kDI = 64;               // indexer dimension of this path
+constexpr int kScanThreads = 256;
+constexpr int kScanRows = 128;        // keys per TMA box (16 per warp)
+constexpr int kScanStages = 8;        // boxes in flight per CTA
+constexpr int kBoxBytes = kScanRows * kDI * 2;
+constexpr int kLaCols = 32;           // linear-state columns per slice
+constexpr int kAttThreads = 256;
+constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kGKeys = 32;            // keys per gather stage
+constexpr int kMaxPer = 2048;         // selected positions per attend CTA
+constexpr int kQRow = kD * 2 + 16;    // padded shared-memory row of a query (bytes)
+constexpr int kCandCap = 256;         // threshold-bin candidates per warp (more: full passes)
+constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
-    int B, n, N_max, H_q, H_kv, group, H_I, M, phi;
-    int KPC;           // keys per CTA (multiple of 16)
-    int ncols;         // linear-state columns per CTA
-    int rowbytes;      // bytes of one cached K (or V) row: H_kv * d * 2
-    float scale_log2;  // sm_scale * log2(e)
+    int B, n, ns, N_max, H_q, H_kv, group, H_I, M, phi;
+    int S1, KPC;        // scan CTAs per sequence, keys per scan CTA
+    int S2, per;        // attend CTAs per sequence, selected positions per attend CTA
+    int la_slices;      // B * H_kv * (kD / kLaCols)
+    int rowbytes;       // bytes of one cached K (or V) row: H_kv * kD * 2
+    float scale_log2;   // sm_scale * log2(e)
     const bf16* q;
     const bf16* k_new;
     const bf16* v_new;
@@ -83,60 +87,20 @@ struct Params {
     bf16* o;
     int32_t* idx;
     int32_t* count;
+    float* scores;      // workspace [B][ns]
+    float* olin;        // workspace [B][H_q][kD]
+    float* part;        // workspace [B][S2][H_q][kD + 2]
+    unsigned* hist;     // workspace [B][4096]: histogram of the top 12 bits of the score keys
     unsigned* status;
-};
-
-// Shared-memory plan (offsets in bytes from a 1024-byte aligned base).
-struct Smem {
-    int region_a;   // TMA ring for the scan, then the K/V gather stages, then partials
-    int scores;     // float[KPC]
-    int hist;       // u32[kMaxBins]    local histogram
-    int bins;       // u32[3][kMaxBins / C]  bin slices this CTA owns, one per pass
-    int s_slice;    // float[128][ncols]
-    int fk;         // float[128]       phi(k_L) of the group's KV head
-    int fq;         // float[16][128]   phi(q_L) of the group's query heads
-    int vcol;       // float[ncols]
-    int zloc;       // float[128]
-    int olin;       // float[16][ncols]
-    int den;        // float[16]
-    int mypos;      // int[kMaxPer]
-    int xchg;       // int[4]   n_gt, n_eq published to the cluster
-    int misc;       // int[64]  broadcasts and per-CTA tables
-    int ctab;       // int[2 * 16 + 16 + 16]
-    int bars;       // uint64[kScanStages + kGStages]
-    int total;
 };
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Smem smem_plan(int C, int KPC, int ncols, int rowbytes, int H_kv) {
-    Smem s;
-    const int scan_bytes = kScanStages * kScanBoxBytes;
-    const int krow = rowbytes + 16;
-    const int gather_bytes = kGStages * kGKeys * 2 * krow;
-    const int part_bytes = H_kv * 16 * (kD + 2) * 4;
-    int a = scan_bytes;
-    if (gather_bytes > a) a = gather_bytes;
-    if (part_bytes > a) a = part_bytes;
-    int off = 0;
-    s.region_a = off; off += align_up(a, 1024);
-    s.scores = off;   off += align_up(KPC * 4, 16);
-    s.hist = off;     off += kMaxBins * 4;
-    s.bins = off;     off += 3 * (kMaxBins / C) * 4;
-    s.s_slice = off;  off += align_up(kD * ncols * 4, 16);
-    s.fk = off;       off += kD * 4;
-    s.fq = off;       off += 16 * kD * 4;
-    s.vcol = off;     off += align_up(ncols * 4, 16);
-    s.zloc = off;     off += kD * 4;
-    s.olin = off;     off += align_up(16 * ncols * 4, 16);
-    s.den = off;      off += 16 * 4;
-    s.mypos = off;    off += kMaxPer * 4;
-    s.xchg = off;     off += 16;
-    s.misc = off;     off += 64 * 4;
-    s.ctab = off;     off += 64 * 4;
-    s.bars = off;     off += (kScanStages + kGStages) * 8;
-    s.total = align_up(off, 16) + 1024;  // slack for aligning the base
-    return s;
+constexpr int kLaThreads = 128;       // linear-branch warps of the scan kernel
+constexpr int kScanBar = 1, kLaBar = 2;  // named barriers of the two warp groups
+
+__device__ __forceinline__ void group_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ float feat(int phi, float x) {
@@ -144,170 +108,233 @@ __device__ __forceinline__ float feat(int phi, float x) {
     return x > 0.0f ? x + 1.0f : __expf(x);
 }
 
-// Exclusive scan over the 256 threads of the block.
-__device__ __forceinline__ int block_scan_excl(int v, int* scratch, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
+// ============================================================================ K1: scan
+struct ScanSmem {
+    static constexpr int ring = 0;                                   // kScanStages boxes
+    static constexpr int s_slice = ring + kScanStages * kBoxBytes;   // float[128][32]
+    static constexpr int fk = s_slice + kD * kLaCols * 4;            // float[128]
+    static constexpr int fq = fk + kD * 4;                           // float[16][128]
+    static constexpr int vcol = fq + 16 * kD * 4;                    // float[32]
+    static constexpr int zloc = vcol + kLaCols * 4;                  // float[128]
+    static constexpr int den = zloc + kD * 4;                        // float[16]
+    static constexpr int stage_sc = den + 16 * 4;                    // float[2][128]
+    static constexpr int lhist = stage_sc + 2 * kScanRows * 4;       // u32[4096]
+    static constexpr int bars = lhist + 4096 * 4;                    // uint64[kScanStages]
+    static constexpr int total = bars + kScanStages * 8 + 1024;      // + base alignment slack
+};
+
+// One slice of the linear branch: sequence b, KV head g, value columns [c0, c0+32).
+// s_slice holds S[:, c0:c0+32] of that head (already loaded).  Run by the
+// kLaThreads threads that follow the scan threads of the block.
+__device__ void linear_slice(const Params& P, int b, int g, int c0, float* s_slice, float* fk,
+                             float* fq, float* vcol, float* zloc, float* den) {
+    const int tid = threadIdx.x - kScanThreads, lane = tid & 31, warp = tid >> 5;
+    const bf16* kl = P.k_L + ((int64_t)b * P.H_kv + g) * kD;
+    const bf16* vl = P.v_L + ((int64_t)b * P.H_kv + g) * kD;
+    // 128-bit loads: 8 bf16 per load, one load per thread for each vector
+    auto unpack8 = [](const uint4& u, float (&f)[8]) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    int off = 0;
-    total = 0;
+        for (int e = 0; e < 4; ++e) {
+            const float2 t = __bfloat1622float2(h2[e]);
+            f[2 * e] = t.x;
+            f[2 * e + 1] = t.y;
+        }
+    };
+    for (int e = tid; e < kD / 8 + kLaCols / 8 + P.group * (kD / 8); e += kLaThreads) {
+        float f[8];
+        if (e < kD / 8) {
+            unpack8(reinterpret_cast<const uint4*>(kl)[e], f);
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        const int x = scratch[w];
-        if (w < warp) off += x;
-        total += x;
+            for (int x = 0; x < 8; ++x) fk[8 * e + x] = feat(P.phi, f[x]);
+        } else if (e < kD / 8 + kLaCols / 8) {
+            const int e2 = e - kD / 8;
+            unpack8(reinterpret_cast<const uint4*>(vl + c0)[e2], f);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) vcol[8 * e2 + x] = f[x];
+        } else {
+            const int e3 = e - kD / 8 - kLaCols / 8;
+            const int h = e3 / (kD / 8), c8 = e3 % (kD / 8);
+            unpack8(reinterpret_cast<const uint4*>(
+                        P.q_L + ((int64_t)b * P.H_q + g * P.group + h) * kD)[c8], f);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) fq[h * kD + 8 * c8 + x] = feat(P.phi, f[x]);
+        }
     }
-    __syncthreads();
-    return off + incl - v;
+    group_sync(kLaBar, kLaThreads);
+    const bool norm = P.phi == LISA_PHI_ELU1_NORM;
+    float* Sg = P.S + ((int64_t)b * P.H_kv + g) * kD * kD;
+    if (norm) {
+        const float* zg = P.z + ((int64_t)b * P.H_kv + g) * kD;
+        for (int i = tid; i < kD; i += kLaThreads) zloc[i] = zg[i] + fk[i];
+    }
+    for (int e = tid; e < kD * kLaCols; e += kLaThreads) {
+        const int i = e / kLaCols, c = e % kLaCols;
+        const float nv = fmaf(fk[i], vcol[c], s_slice[e]);
+        s_slice[e] = nv;
+        Sg[(int64_t)i * kD + c0 + c] = nv;
+    }
+    group_sync(kLaBar, kLaThreads);
+    if (norm) {
+        // z itself is advanced by the attend kernel: the sibling slices of this
+        // head still read the old z here
+        for (int h = warp; h < P.group; h += kLaThreads / 32) {
+            float dz = 0.0f;
+            for (int i = lane; i < kD; i += 32) dz = fmaf(fq[h * kD + i], zloc[i], dz);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dz += __shfl_xor_sync(0xffffffffu, dz, o);
+            if (lane == 0) den[h] = dz;
+        }
+        group_sync(kLaBar, kLaThreads);
+    }
+    for (int e = tid; e < P.group * kLaCols; e += kLaThreads) {
+        const int h = e / kLaCols, c = e % kLaCols;
+        float acc = 0.0f;
+#pragma unroll 8
+        for (int i = 0; i < kD; ++i) acc = fmaf(fq[h * kD + i], s_slice[i * kLaCols + c], acc);
+        P.olin[((int64_t)b * P.H_q + g * P.group + h) * kD + c0 + c] = norm ? acc / den[h] : acc;
+    }
+    group_sync(kLaBar, kLaThreads);
 }
 
-template <int C>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_decode_fused(const __grid_constant__ CUtensorMap tmap_kI, const Params P) {
+__global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
+    k_decode_scan(const __grid_constant__ CUtensorMap tmap_kI, const Params P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const Smem L = smem_plan(C, P.KPC, P.ncols, P.rowbytes, P.H_kv);
-    uint8_t* region_a = base + L.region_a;
-    float* scores = reinterpret_cast<float*>(base + L.scores);
-    uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.hist);
-    uint32_t* bins = reinterpret_cast<uint32_t*>(base + L.bins);
-    float* s_slice = reinterpret_cast<float*>(base + L.s_slice);
-    float* fk = reinterpret_cast<float*>(base + L.fk);
-    float* fq = reinterpret_cast<float*>(base + L.fq);
-    float* vcol = reinterpret_cast<float*>(base + L.vcol);
-    float* zloc = reinterpret_cast<float*>(base + L.zloc);
-    float* olin = reinterpret_cast<float*>(base + L.olin);
-    float* den = reinterpret_cast<float*>(base + L.den);
-    int* mypos = reinterpret_cast<int*>(base + L.mypos);
-    int* xchg = reinterpret_cast<int*>(base + L.xchg);
-    int* misc = reinterpret_cast<int*>(base + L.misc);
-    int* ctab = reinterpret_cast<int*>(base + L.ctab);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bars);
-    uint64_t* scan_bar = bars;
-    uint64_t* gath_bar = bars + kScanStages;
+    uint8_t* ring = base + ScanSmem::ring;
+    float* s_slice = reinterpret_cast<float*>(base + ScanSmem::s_slice);
+    float* fk = reinterpret_cast<float*>(base + ScanSmem::fk);
+    float* fq = reinterpret_cast<float*>(base + ScanSmem::fq);
+    float* vcol = reinterpret_cast<float*>(base + ScanSmem::vcol);
+    float* zloc = reinterpret_cast<float*>(base + ScanSmem::zloc);
+    float* den = reinterpret_cast<float*>(base + ScanSmem::den);
+    float* stage_sc = reinterpret_cast<float*>(base + ScanSmem::stage_sc);
+    unsigned* lhist = reinterpret_cast<unsigned*>(base + ScanSmem::lhist);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + ScanSmem::bars);
 
+    ptx::pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
-    const int r = (int)ptx::cluster_ctarank();
-    const int b = blockIdx.x / C;
+    const int b = blockIdx.x / P.S1, j = blockIdx.x % P.S1;
     const int n = P.n, p = n - 1;
-    const int k0 = r * P.KPC;
+    const int k0 = j * P.KPC;
     const int k1 = min(n, k0 + P.KPC);
     const int nk = max(0, k1 - k0);
-    const int n_scan_stages = (nk + kScanRows - 1) / kScanRows;
-    const int per_owner = kMaxBins / C;
-    bool ok = true;  // false once a bounded wait gave up
+    const int nst = (nk + kScanRows - 1) / kScanRows;
+    bool ok = true;
 
-    // ---------------------------------------------------------------- set-up
     if (tid == 0) {
-        for (int i = 0; i < kScanStages + kGStages; ++i) ptx::mbar_init(&bars[i], 1);
+        for (int i = 0; i < kScanStages; ++i) ptx::mbar_init(&bars[i], 1);
         ptx::fence_mbar_init();
-    }
-    for (int i = tid; i < 3 * per_owner; i += kThreads) bins[i] = 0;
-    __syncthreads();
-    // First cluster barrier: every CTA's bins are zero and its shared memory is
-    // live before anyone touches it remotely.  Waited on before the first
-    // remote access, so the scan overlaps it.
-    ptx::cluster_arrive();
-
-    if (tid == 0) {
-        const int first = min(n_scan_stages, kScanStages);
-        for (int st = 0; st < first; ++st) {
-            ptx::mbar_arrive_expect_tx(&scan_bar[st], kScanBoxBytes);
-            ptx::tma_load_2d(region_a + st * kScanBoxBytes, &tmap_kI, 0,
-                             b * P.N_max + k0 + st * kScanRows, &scan_bar[st]);
+        for (int st = 0; st < min(nst, kScanStages); ++st) {
+            ptx::mbar_arrive_expect_tx(&bars[st], kBoxBytes);
+            ptx::tma_load_2d(ring + st * kBoxBytes, &tmap_kI, 0, b * P.N_max + k0 + st * kScanRows,
+                             &bars[st]);
         }
     }
-    // Linear-state slice of this CTA: KV head g_r, columns [c0, c0 + ncols).
-    const int cta_per_head = C / P.H_kv;
-    const int g_r = r / cta_per_head;
-    const int c0 = (r % cta_per_head) * P.ncols;
-    float* Sg = P.S + ((int64_t)b * P.H_kv + g_r) * kD * kD;
-    {
-        const int chunks_per_row = P.ncols / 4;
-        for (int e = tid; e < kD * chunks_per_row; e += kThreads) {
-            const int i = e / chunks_per_row, c = (e % chunks_per_row) * 4;
-            ptx::cp_async_16(s_slice + i * P.ncols + c, Sg + (int64_t)i * kD + c0 + c);
+    // prefetch this CTA's first linear-state slice
+    const int slice = blockIdx.x;
+    const int slices_per_b = P.H_kv * (kD / kLaCols);
+    const bool la_thread = tid >= kScanThreads;
+    if (la_thread && slice < P.la_slices) {
+        const int lb = slice / slices_per_b, lg = (slice / (kD / kLaCols)) % P.H_kv;
+        const int lc0 = (slice % (kD / kLaCols)) * kLaCols;
+        const float* Sg = P.S + ((int64_t)lb * P.H_kv + lg) * kD * kD;
+        for (int e = tid - kScanThreads; e < kD * kLaCols / 4; e += kLaThreads) {
+            const int i = e / (kLaCols / 4), c = (e % (kLaCols / 4)) * 4;
+            ptx::cp_async_16(s_slice + i * kLaCols + c, Sg + (int64_t)i * kD + lc0 + c);
         }
         ptx::cp_async_commit();
     }
-    // Cache append of the new token (nobody in this launch reads row p of the
-    // caches: the scan and the gather take it from the inputs).
-    if (r == 0) {
-        const int kv_chunks = P.rowbytes / 16;
+    __syncthreads();  // barriers initialised; from here the two warp groups run apart
+    if (la_thread) {
+        if (slice < P.la_slices) {
+            ptx::cp_async_wait_all();
+            group_sync(kLaBar, kLaThreads);
+            const int lb = slice / slices_per_b, lg = (slice / (kD / kLaCols)) % P.H_kv;
+            const int lc0 = (slice % (kD / kLaCols)) * kLaCols;
+            linear_slice(P, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
+        }
+        for (int sl = slice + gridDim.x; sl < P.la_slices; sl += gridDim.x) {
+            const int lb = sl / slices_per_b, lg = (sl / (kD / kLaCols)) % P.H_kv;
+            const int lc0 = (sl % (kD / kLaCols)) * kLaCols;
+            const float* Sg = P.S + ((int64_t)lb * P.H_kv + lg) * kD * kD;
+            for (int e = tid - kScanThreads; e < kD * kLaCols; e += kLaThreads)
+                s_slice[e] = Sg[(int64_t)(e / kLaCols) * kD + lc0 + e % kLaCols];
+            group_sync(kLaBar, kLaThreads);
+            linear_slice(P, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
+        }
+        return;
+    }
+    if (j == 0) {
+        // cache append of the new token (K2 reads row p from the inputs, not the cache)
+        const int chunks = P.rowbytes / 16;
         const uint4* kn = reinterpret_cast<const uint4*>(P.k_new + (int64_t)b * P.H_kv * kD);
         const uint4* vn = reinterpret_cast<const uint4*>(P.v_new + (int64_t)b * P.H_kv * kD);
         uint4* kd = reinterpret_cast<uint4*>(P.k_cache + ((int64_t)b * P.N_max + p) * P.H_kv * kD);
         uint4* vd = reinterpret_cast<uint4*>(P.v_cache + ((int64_t)b * P.N_max + p) * P.H_kv * kD);
-        for (int i = tid; i < kv_chunks; i += kThreads) {
+        for (int i = tid; i < chunks; i += kScanThreads) {
             kd[i] = kn[i];
             vd[i] = vn[i];
         }
         if (tid < kDI / 8) {
             const uint4* kin = reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * kDI);
-            uint4* kid = reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * kDI);
-            kid[tid] = kin[tid];
+            reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * kDI)[tid] = kin[tid];
         }
     }
+    for (int i = tid; i < 4096; i += kScanThreads) lhist[i] = 0u;
 
-    // ---------------------------------------------------------------- A: indexer scan
-    // Fragment layout (mma m16n8k16, A = 16 keys x 16 dims, B = 16 dims x 8 heads):
-    // the thread (gid, tq) holds dims [16 tq, 16 tq + 16) of its rows; k-step s
-    // uses dims 16 tq + 4 s + {0,1} and {2,3}.  A and B use the same dim order,
-    // so the dot products are unchanged.
+    // Indexer fragments.  mma m16n8k16 with A = 16 keys x 16 dims and B = 16 dims
+    // x 8 heads; the thread (gid, tq) holds dims [16 tq, 16 tq + 16) of its rows
+    // and k-step s uses dims 16 tq + 4 s + {0,1} / {2,3}: A and B share this dim
+    // order, so every dot product is unchanged.
     uint32_t qb[8];
     float w_lo = 0.0f, w_hi = 0.0f;
-    {
-        if (gid < P.H_I) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                P.q_I + ((int64_t)b * P.H_I + gid) * kDI + 16 * tq);
-            const uint4 u0 = src[0], u1 = src[1];
-            qb[0] = u0.x; qb[1] = u0.y; qb[2] = u0.z; qb[3] = u0.w;
-            qb[4] = u1.x; qb[5] = u1.y; qb[6] = u1.z; qb[7] = u1.w;
-        } else {
+    if (gid < P.H_I) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(P.q_I + ((int64_t)b * P.H_I + gid) * kDI + 16 * tq);
+        const uint4 u0 = src[0], u1 = src[1];
+        qb[0] = u0.x; qb[1] = u0.y; qb[2] = u0.z; qb[3] = u0.w;
+        qb[4] = u1.x; qb[5] = u1.y; qb[6] = u1.z; qb[7] = u1.w;
+    } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) qb[i] = 0u;
-        }
+        for (int i = 0; i < 8; ++i) qb[i] = 0u;
+    }
+    {
         const float* wb = P.w + (int64_t)b * P.H_I;
         if (2 * tq < P.H_I) w_lo = wb[2 * tq];
         if (2 * tq + 1 < P.H_I) w_hi = wb[2 * tq + 1];
     }
-    for (int st = 0; st < n_scan_stages; ++st) {
+    float* srow = P.scores + (int64_t)b * P.ns;
+    for (int st = 0; st < nst; ++st) {
         const int buf = st % kScanStages;
-        const uint32_t parity = (st / kScanStages) & 1;
-        if (ok && !ptx::mbar_wait_bounded(&scan_bar[buf], parity, kWaitTries)) {
+        if (ok && !ptx::mbar_wait_bounded(&bars[buf], (st / kScanStages) & 1, kWaitTries)) {
             ok = false;
             if (tid == 0) record_error(P.status, kDevTimeout);
         }
+        float* ssc = stage_sc + (st & 1) * kScanRows;
         if (ok) {
-            const uint8_t* tile = region_a + buf * kScanBoxBytes;
+            const uint8_t* tile = ring + buf * kBoxBytes;
             const int row0 = warp * 16 + gid;
             uint32_t ra[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = row0 + 8 * h;
-                const int pos = k0 + st * kScanRows + row;
-                if (pos == p) {
-                    const uint4* src = reinterpret_cast<const uint4*>(
-                        P.k_I_new + (int64_t)b * kDI + 16 * tq);
-                    const uint4 u0 = src[0], u1 = src[1];
-                    ra[h][0] = u0.x; ra[h][1] = u0.y; ra[h][2] = u0.z; ra[h][3] = u0.w;
-                    ra[h][4] = u1.x; ra[h][5] = u1.y; ra[h][6] = u1.z; ra[h][7] = u1.w;
+                uint4 u0, u1;
+                if (k0 + st * kScanRows + row == p) {
+                    const uint4* src =
+                        reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * kDI + 16 * tq);
+                    u0 = src[0];
+                    u1 = src[1];
                 } else {
                     const uint8_t* rp = tile + row * 128;
                     const int sw = row & 7;
-                    const uint4 u0 = *reinterpret_cast<const uint4*>(rp + (((2 * tq) ^ sw) << 4));
-                    const uint4 u1 = *reinterpret_cast<const uint4*>(rp + (((2 * tq + 1) ^ sw) << 4));
-                    ra[h][0] = u0.x; ra[h][1] = u0.y; ra[h][2] = u0.z; ra[h][3] = u0.w;
-                    ra[h][4] = u1.x; ra[h][5] = u1.y; ra[h][6] = u1.z; ra[h][7] = u1.w;
+                    u0 = *reinterpret_cast<const uint4*>(rp + (((2 * tq) ^ sw) << 4));
+                    u1 = *reinterpret_cast<const uint4*>(rp + (((2 * tq + 1) ^ sw) << 4));
                 }
+                ra[h][0] = u0.x; ra[h][1] = u0.y; ra[h][2] = u0.z; ra[h][3] = u0.w;
+                ra[h][4] = u1.x; ra[h][5] = u1.y; ra[h][6] = u1.z; ra[h][7] = u1.w;
             }
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -321,436 +348,569 @@ __global__ void __launch_bounds__(kThreads, 1)
             s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-            const int lr0 = st * kScanRows + row0;  // local key index
-            if (tq == 0 && lr0 < nk) scores[lr0] = s0;
-            if (tq == 1 && lr0 + 8 < nk) scores[lr0 + 8] = s1;
+            if (tq == 0) ssc[row0] = s0;
+            if (tq == 1) ssc[row0 + 8] = s1;
         }
-        __syncthreads();  // every warp is done with this buffer
-        if (tid == 0 && ok && st + kScanStages < n_scan_stages) {
-            ptx::mbar_arrive_expect_tx(&scan_bar[buf], kScanBoxBytes);
-            ptx::tma_load_2d(region_a + buf * kScanBoxBytes, &tmap_kI, 0,
-                             b * P.N_max + k0 + (st + kScanStages) * kScanRows, &scan_bar[buf]);
+        group_sync(kScanBar, kScanThreads);  // box consumed; this stage's scores in shared memory
+        if (tid == 0 && ok && st + kScanStages < nst) {
+            ptx::mbar_arrive_expect_tx(&bars[buf], kBoxBytes);
+            ptx::tma_load_2d(ring + buf * kBoxBytes, &tmap_kI, 0,
+                             b * P.N_max + k0 + (st + kScanStages) * kScanRows, &bars[buf]);
         }
+        if (ok && tid < kScanRows) {
+            const int pos = k0 + st * kScanRows + tid;
+            if (pos < k1) {
+                const float v = ssc[tid];
+                srow[pos] = v;
+                atomicAdd(&lhist[order_key(v) >> 20], 1u);
+            }
+        }
+    }
+    // this slice's part of the sequence's 12-bit key histogram
+    group_sync(kScanBar, kScanThreads);
+    for (int i = tid; i < 4096; i += kScanThreads) {
+        const unsigned v = lhist[i];
+        if (v) atomicAdd(&P.hist[(int64_t)b * 4096 + i], v);
     }
 
-    // ---------------------------------------------------------------- A': linear branch
-    ptx::cp_async_wait_all();
-    {
-        const bf16* kl = P.k_L + ((int64_t)b * P.H_kv + g_r) * kD;
-        const bf16* vl = P.v_L + ((int64_t)b * P.H_kv + g_r) * kD;
-        for (int i = tid; i < kD; i += kThreads) {
-            fk[i] = feat(P.phi, __bfloat162float(kl[i]));
-        }
-        for (int c = tid; c < P.ncols; c += kThreads) vcol[c] = __bfloat162float(vl[c0 + c]);
-        for (int e = tid; e < P.group * kD; e += kThreads) {
-            const int h = e / kD, i = e % kD;
-            fq[h * kD + i] =
-                feat(P.phi, __bfloat162float(P.q_L[((int64_t)b * P.H_q + g_r * P.group + h) * kD + i]));
-        }
+    if (!ok && tid == 0) {
+        // give copies still in flight a bounded chance to land before exit
+        for (int i = 0; i < kScanStages; ++i)
+            for (uint32_t par = 0; par < 2; ++par) ptx::mbar_wait_bounded(&bars[i], par, 1u << 16);
     }
-    __syncthreads();
-    const bool norm = P.phi == LISA_PHI_ELU1_NORM;
-    if (norm) {
-        const float* zg = P.z + ((int64_t)b * P.H_kv + g_r) * kD;
-        for (int i = tid; i < kD; i += kThreads) zloc[i] = zg[i] + fk[i];
-    }
-    for (int e = tid; e < kD * P.ncols; e += kThreads) {
-        const int i = e / P.ncols, c = e % P.ncols;
-        const float nv = fmaf(fk[i], vcol[c], s_slice[e]);
-        s_slice[e] = nv;
-        Sg[(int64_t)i * kD + c0 + c] = nv;
-    }
-    __syncthreads();
-    if (norm) {
-        if (c0 == 0)
-            for (int i = tid; i < kD; i += kThreads)
-                P.z[((int64_t)b * P.H_kv + g_r) * kD + i] = zloc[i];
-        for (int h = warp; h < P.group; h += kWarps) {
-            float dz = 0.0f;
-            for (int i = lane; i < kD; i += 32) dz = fmaf(fq[h * kD + i], zloc[i], dz);
+}
+
+// ============================================================================ K2: attend
+template <int HKV>
+struct Att {
+    static constexpr int rowbytes = HKV * kD * 2;     // one cached K (or V) row
+    static constexpr int krow = rowbytes + 16;        // padded shared-memory row
+    static constexpr int rpc = rowbytes / 16;         // 16-byte chunks per row
+    static constexpr int stage_bytes = kGKeys * 2 * krow;
+    static constexpr int chunks_per_thread = kGKeys * 2 * rpc / kAttThreads;
+    static constexpr int wph = kAttWarps / HKV;       // warps per KV head
+    static constexpr int dw = kD / wph;               // output dims per warp
+    static constexpr int ntile_o = dw / 8;
+    // shared memory: histogram, broadcasts, selected positions, queries, stages
+    static constexpr int hist = 0;                     // two 2048-bin halves (warps 0-3, 4-7)
+    static constexpr int bar = hist + 2 * 2048 * 4;
+    static constexpr int bc = bar + 16;                 // int[128]: broadcasts, scratch
+    static constexpr int mypos = bc + 128 * 4;
+    static constexpr int q = mypos + kMaxPer * 4;
+    static constexpr int cand = q + ((HKV * 16 * kQRow + 127) / 128) * 128;  // uint2[8][kCandCap]
+    static constexpr int stage = cand + kAttWarps * kCandCap * 8;
+    static constexpr int total = stage + 2 * stage_bytes;
+    static constexpr int key_cap = 2 * stage_bytes / 4 - 32;  // scores that fit in the stages
+};
+
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dz += __shfl_xor_sync(0xffffffffu, dz, o);
-            if (lane == 0) den[h] = dz;
-        }
-        __syncthreads();
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
     }
-    for (int e = tid; e < P.group * P.ncols; e += kThreads) {
-        const int h = e / P.ncols, c = e % P.ncols;
-        float acc = 0.0f;
-        for (int i = 0; i < kD; ++i) acc = fmaf(fq[h * kD + i], s_slice[i * P.ncols + c], acc);
-        olin[h * P.ncols + c] = norm ? acc / den[h] : acc;
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    int off = 0;
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) {
+        const int x = scratch[w];
+        if (w < warp) off += x;
+        total += x;
     }
+    __syncthreads();
+    return off + incl - v;
+}
 
-    // ---------------------------------------------------------------- B: top-M
-    ptx::cluster_wait();  // matches the set-up arrive
+template <int HKV>
+__global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P) {
+    using A = Att<HKV>;
+    extern __shared__ __align__(128) uint8_t att_raw[];
+    unsigned* hist = reinterpret_cast<unsigned*>(att_raw + A::hist);
+    uint64_t* rowbar = reinterpret_cast<uint64_t*>(att_raw + A::bar);
+    int* bc = reinterpret_cast<int*>(att_raw + A::bc);
+    int* scratch = bc + 32;
+    int* mypos = reinterpret_cast<int*>(att_raw + A::mypos);
+    uint8_t* qs = att_raw + A::q;
+    uint8_t* stage = att_raw + A::stage;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tq = lane & 3;
+    const int b = blockIdx.x / P.S2, j = blockIdx.x % P.S2;
+    const int n = P.n, p = n - 1;
+    ptx::pdl_launch_dependents();
+
+    // ---- prologue (inputs only; nothing written by the scan kernel)
+    for (int e = tid; e < HKV * 16 * (kD / 8); e += kAttThreads) {
+        const int g = e / (16 * (kD / 8)), r = (e / (kD / 8)) % 16, c = e % (kD / 8);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < P.group)
+            v = reinterpret_cast<const uint4*>(P.q + ((int64_t)b * P.H_q + g * P.group + r) * kD)[c];
+        *reinterpret_cast<uint4*>(qs + (g * 16 + r) * kQRow + c * 16) = v;
+    }
+    if (tid == 0) {
+        ptx::mbar_init(rowbar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    ptx::pdl_wait_prior();  // scores, histogram and linear output of this call are ready
+
+    // ---- exact top-M of the score row (the same result in every CTA of the sequence)
+    // Radix select on the 32-bit order-preserving key of each score, most
+    // significant digit first: 12 bits (the histogram the scan kernel built),
+    // then 10 and 10 bits over the keys that share the digits found so far.
+    // Ties at the M-th key keep the lowest positions.
+    const float* srow = P.scores + (int64_t)b * P.ns;
     const int cnt = min(P.M, n);
-    int* scan_scratch = misc;       // [kWarps]
-    int* bc = misc + 16;            // broadcasts
-    int sel_offset = 0, n_sel = 0;  // this CTA's selected positions and their global offset
-    uint32_t tau = 0;
-    int krem = 0;
-    int my_take_eq = 0;  // keys equal to the threshold this CTA keeps (lowest positions first)
-    const bool select_all = n <= P.M;
-    if (!select_all) {
-        uint32_t prefix = 0, mask = 0;
-        krem = P.M;
-        for (int pass = 0; pass < 3; ++pass) {
-            const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-            const int nb = pass == 2 ? 1024 : 2048;
-            const int owner_span = nb / C;
-            for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
-            __syncthreads();
-            for (int i = tid; i < nk; i += kThreads) {
-                const uint32_t key = order_key(scores[i]);
-                if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-            }
-            __syncthreads();
-            uint32_t* pass_bins = bins + pass * per_owner;
-            for (int i = tid; i < nb; i += kThreads) {
-                const uint32_t v = hist[i];
-                if (v) {
-                    const uint32_t owner = i / owner_span;
-                    const uint32_t addr = ptx::mapa(ptx::smem_u32(pass_bins + (i % owner_span)), owner);
-                    ptx::red_add_dsmem_u32(addr, v);
-                }
-            }
-            ptx::cluster_sync();
-            // Every CTA reads the whole histogram: thread t owns bins [t*bpt, (t+1)*bpt).
-            const int bpt = nb / kThreads;  // 8 or 4
-            uint32_t hv[8];
-            int tsum = 0;
-            for (int j = 0; j < bpt; ++j) {
-                const int i = tid * bpt + j;
-                const uint32_t owner = i / owner_span;
-                hv[j] = ptx::ld_dsmem_u32(ptx::mapa(ptx::smem_u32(pass_bins + (i % owner_span)), owner));
-                tsum += (int)hv[j];
-            }
-            // suffix sum over threads (bins above this thread's range)
+    const int lo = j * P.per, hi = min(cnt, lo + P.per);
+    const int mine = max(0, hi - lo);
+    if (n <= P.M) {
+        for (int i = tid; i < mine; i += kAttThreads) mypos[i] = lo + i;
+    } else {
+        float* srow_s = reinterpret_cast<float*>(stage);
+        const bool resident = n <= A::key_cap;
+        bool row_ok = true;
+        if (resident && tid == 0) {
+            const int bytes = ((n + 3) / 4) * 16;
+            ptx::mbar_arrive_expect_tx(rowbar, bytes);
+            for (int off = 0; off < bytes; off += 16384)
+                ptx::bulk_load(stage + off, srow + off / 4, min(16384, bytes - off), rowbar);
+        }
+        // first digit from the sequence histogram (while the row is in flight)
+        auto find_bin = [&](const unsigned* hv, int bpt, int tsum, int need) {
             int total;
-            const int below = block_scan_excl(tsum, scan_scratch, total);
+            const int below = block_excl_scan(tsum, scratch, total);
             const int above = total - below - tsum;
-            if (above < krem && krem <= above + tsum) {
+            if (tid == 0) { bc[0] = 0; bc[1] = 1; }
+            __syncthreads();
+            if (above < need && need <= above + tsum) {
                 int acc = above;
-                for (int j = bpt - 1; j >= 0; --j) {
-                    if (acc + (int)hv[j] >= krem) {
-                        bc[0] = tid * bpt + j;
-                        bc[1] = krem - acc;
+                for (int q = bpt - 1; q >= 0; --q) {
+                    if (acc + (int)hv[q] >= need) {
+                        bc[0] = tid * bpt + q;
+                        bc[1] = need - acc;
                         break;
                     }
-                    acc += (int)hv[j];
+                    acc += (int)hv[q];
                 }
             }
             __syncthreads();
+        };
+        uint32_t b1;
+        int krem;
+        {
+            unsigned hv[16];
+            int tsum = 0;
+            const uint4* g4 = reinterpret_cast<const uint4*>(P.hist + (int64_t)b * 4096) + tid * 4;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 u = __ldcg(g4 + q);
+                hv[4 * q] = u.x; hv[4 * q + 1] = u.y; hv[4 * q + 2] = u.z; hv[4 * q + 3] = u.w;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) tsum += (int)hv[q];
+            find_bin(hv, 16, tsum, P.M);
+            b1 = (uint32_t)bc[0];
+            krem = bc[1];
+        }
+        if (resident && !ptx::mbar_wait_bounded(rowbar, 0, kWaitTries)) {
+            row_ok = false;
+            if (tid == 0) record_error(P.status, kDevTimeout);
+        }
+        const float* rsrc = resident ? srow_s : srow;
+        auto keys8 = [&](int base, uint32_t (&k)[8]) {
+            const float4* src = reinterpret_cast<const float4*>(rsrc) + base / 4;
+            float4 v0, v1;
+            if (resident) { v0 = src[0]; v1 = src[1]; }
+            else { v0 = __ldcg(src); v1 = __ldcg(src + 1); }
+            k[0] = order_key(v0.x); k[1] = order_key(v0.y); k[2] = order_key(v0.z); k[3] = order_key(v0.w);
+            k[4] = order_key(v1.x); k[5] = order_key(v1.y); k[6] = order_key(v1.z); k[7] = order_key(v1.w);
+        };
+        auto warp_excl = [&](int v, int& tot) {
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            tot = __shfl_sync(0xffffffffu, incl, 31);
+            return incl - v;
+        };
+        // Warp w owns positions [w*seg, (w+1)*seg), walked in blocks of 256 with
+        // lane l on the 8 consecutive positions blk + 8l .. blk + 8l + 7.
+        const int seg = ((n + kAttWarps - 1) / kAttWarps + 255) / 256 * 256;
+        const int s0 = warp * seg, s1 = min(n, s0 + seg);
+        uint2* clist = reinterpret_cast<uint2*>(att_raw + A::cand) + warp * kCandCap;
+        // scan A: keys above the first digit, and the threshold-digit candidates (in order)
+        int n_above = 0, ncand = 0;
+        if (row_ok) {
+#pragma unroll 1
+            for (int blk = s0; blk < s1; blk += 256) {
+                const int base = blk + lane * 8;
+                uint32_t k[8];
+                unsigned cm = 0;
+                if (base < s1) {
+                    keys8(base, k);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const bool v = base + e < s1;
+                        n_above += v && (k[e] >> 20) > b1;
+                        cm |= (unsigned)(v && (k[e] >> 20) == b1) << e;
+                    }
+                }
+                int ctot;
+                int w = ncand + warp_excl(__popc(cm), ctot);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if ((cm >> e) & 1u) {
+                        if (w < kCandCap) clist[w] = make_uint2(k[e], (uint32_t)(base + e));
+                        ++w;
+                    }
+                ncand += ctot;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
+        if (lane == 0) { scratch[8 + warp] = n_above; scratch[16 + warp] = ncand; }
+        __syncthreads();
+        bool overflow = false;
+        for (int w = 0; w < kAttWarps; ++w) overflow |= scratch[16 + w] > kCandCap;
+        // refine: 10 bits, then 10 bits, over the candidates (or, if a warp's
+        // list overflowed, over every key of the row with the first digit b1)
+        uint32_t prefix = b1 << 20, mask = 0xFFFu << 20;
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0;
+            for (int i = tid; i < 1024; i += kAttThreads) hist[i] = 0u;
+            __syncthreads();
+            if (row_ok) {
+                if (!overflow) {
+                    for (int i = tid; i < kAttWarps * kCandCap; i += kAttThreads) {
+                        const int w = i / kCandCap, c = i % kCandCap;
+                        if (c < scratch[16 + w]) {
+                            const uint32_t k = reinterpret_cast<const uint2*>(att_raw + A::cand)[i].x;
+                            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 1023u], 1u);
+                        }
+                    }
+                } else {
+                    for (int i8 = tid * 8; i8 < n; i8 += kAttThreads * 8) {
+                        uint32_t k[8];
+                        keys8(i8, k);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (i8 + e < n && (k[e] & mask) == prefix)
+                                atomicAdd(&hist[(k[e] >> shift) & 1023u], 1u);
+                    }
+                }
+            }
+            __syncthreads();
+            unsigned hv[4];
+            int tsum = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) { hv[q] = hist[tid * 4 + q]; tsum += (int)hv[q]; }
+            find_bin(hv, 4, tsum, krem);
             prefix |= (uint32_t)bc[0] << shift;
             krem = bc[1];
-            mask |= (uint32_t)(nb - 1) << shift;
+            mask |= 1023u << shift;
             __syncthreads();
         }
-        tau = prefix;
-        // local counts above and equal to the threshold
-        if (tid == 0) { bc[2] = 0; bc[3] = 0; }
-        __syncthreads();
-        int gt = 0, eq = 0;
-        for (int i = tid; i < nk; i += kThreads) {
-            const uint32_t key = order_key(scores[i]);
-            gt += key > tau;
-            eq += key == tau;
-        }
-        if (gt) atomicAdd(&bc[2], gt);
-        if (eq) atomicAdd(&bc[3], eq);
-        __syncthreads();
-        if (tid == 0) { xchg[0] = bc[2]; xchg[1] = bc[3]; }
-        ptx::cluster_sync();
-        if (tid < C) {
-            ctab[tid] = (int)ptx::ld_dsmem_u32(ptx::mapa(ptx::smem_u32(xchg), tid));
-            ctab[16 + tid] = (int)ptx::ld_dsmem_u32(ptx::mapa(ptx::smem_u32(xchg + 1), tid));
-        }
-        __syncthreads();
-        // ties: the lowest positions win, so CTAs take their equal keys in rank order
-        int eq_before = 0, off = 0;
-        for (int c = 0; c < C; ++c) {
-            const int take = max(0, min(ctab[16 + c], krem - eq_before));
-            const int sel = ctab[c] + take;
-            if (c == r) { sel_offset = off; n_sel = sel; my_take_eq = take; }
-            eq_before += ctab[16 + c];
-            off += sel;
-        }
-    } else {
-        sel_offset = k0;
-        n_sel = nk;
-    }
-
-    // Ordered compaction of this CTA's selected keys into the owners' lists.
-    const int per = (cnt + C - 1) / C;
-    {
-        const int kpt = (nk + kThreads - 1) / kThreads;
-        const int i0 = tid * kpt, i1 = min(nk, i0 + kpt);
-        const int take_eq = my_take_eq;
-        int eq_rank0 = 0;
-        // rank of this thread's first equal key among the CTA's equal keys
-        int my_eq = 0;
-        if (!select_all)
-            for (int i = i0; i < i1; ++i) my_eq += order_key(scores[i]) == tau;
-        int tot_eq;
-        eq_rank0 = block_scan_excl(my_eq, scan_scratch, tot_eq);
-        int my_sel = 0;
-        {
-            int er = eq_rank0;
-            for (int i = i0; i < i1; ++i) {
-                if (select_all) { ++my_sel; continue; }
-                const uint32_t key = order_key(scores[i]);
-                if (key > tau) ++my_sel;
-                else if (key == tau) { if (er < take_eq) ++my_sel; ++er; }
+        const uint32_t tau = prefix;  // the M-th largest key; krem of its ties are kept
+        // selected count of each warp's segment: keys above b1, plus candidates
+        // above tau, plus the ties that fall to it in position order
+        int gt_c = 0, eq_c = 0;
+        if (!overflow) {
+            for (int c = lane; c < scratch[16 + warp]; c += 32) {
+                const uint32_t k = clist[c].x;
+                gt_c += k > tau;
+                eq_c += k == tau;
+            }
+        } else if (row_ok) {
+            for (int blk = s0; blk < s1; blk += 256) {
+                const int base = blk + lane * 8;
+                if (base >= s1) continue;
+                uint32_t k[8];
+                keys8(base, k);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (base + e < s1 && (k[e] >> 20) == b1) { gt_c += k[e] > tau; eq_c += k[e] == tau; }
             }
         }
-        int tot_sel;
-        int rank = block_scan_excl(my_sel, scan_scratch, tot_sel);
-        int er = eq_rank0;
-        for (int i = i0; i < i1; ++i) {
-            bool sel;
-            if (select_all) {
-                sel = true;
-            } else {
-                const uint32_t key = order_key(scores[i]);
-                sel = key > tau;
-                if (key == tau) { sel = er < take_eq; ++er; }
-            }
-            if (!sel) continue;
-            const int gi = sel_offset + rank++;
-            const int pos = k0 + i;
-            const int dest = gi / per, slot = gi - dest * per;
-            ptx::st_dsmem_u32(ptx::mapa(ptx::smem_u32(mypos + slot), dest), (uint32_t)pos);
-            if (P.idx) P.idx[(int64_t)b * P.M + gi] = pos;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            gt_c += __shfl_xor_sync(0xffffffffu, gt_c, o);
+            eq_c += __shfl_xor_sync(0xffffffffu, eq_c, o);
         }
-        (void)n_sel;
-        if (P.idx && r == 0)
-            for (int i = cnt + tid; i < P.M; i += kThreads) P.idx[(int64_t)b * P.M + i] = -1;
-        if (P.count && r == 0 && tid == 0) P.count[b] = cnt;
-    }
-    ptx::cluster_sync();  // every CTA's list is complete
-
-    // ---------------------------------------------------------------- C: gather + attention
-    const int my_cnt = max(0, min(cnt - r * per, per));
-    const int wph = kWarps / P.H_kv;  // warps per KV head
-    const int g_w = warp / wph;
-    const int part = warp % wph;
-    const int dw = kD / wph;          // output dims of this warp
-    const int krow = P.rowbytes + 16;
-    const int stage_bytes = kGKeys * 2 * krow;
-    // query fragments of head group g_w: rows = query heads (group <= 16), 8 k-steps
-    uint32_t qa[8][4];
-    {
-        const int h0 = g_w * P.group;
+        if (lane == 0) { scratch[24 + warp] = gt_c; scratch[32 + warp] = eq_c; }
+        __syncthreads();
+        int eq_before = 0, sel_before = 0;
+        for (int w = 0; w < warp; ++w) {
+            const int eqw = scratch[32 + w];
+            sel_before += scratch[8 + w] + scratch[24 + w] + max(0, min(eqw, krem - eq_before));
+            eq_before += eqw;
+        }
+        const int sel_w = n_above + gt_c + max(0, min(eq_c, krem - eq_before));
+        // ranked walk, only where this warp's ranks meet this CTA's share [lo, hi)
+        if (row_ok && sel_before < hi && sel_before + sel_w > lo) {
+            const unsigned lt_all = 0xffffffffu;
+#pragma unroll 1
+            for (int blk = s0; blk < s1; blk += 256) {
+                const int base = blk + lane * 8;
+                uint32_t k[8];
+                unsigned eqm = 0, selm = 0;
+                if (base < s1) {
+                    keys8(base, k);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = gid + 8 * hh;
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    uint32_t v = 0u;
-                    if (row < P.group)
-                        v = *reinterpret_cast<const uint32_t*>(
-                            P.q + ((int64_t)b * P.H_q + h0 + row) * kD + ks * 16 + 2 * tq + 8 * kk);
-                    qa[ks][hh + 2 * kk] = v;
+                    for (int e = 0; e < 8; ++e) {
+                        const bool v = base + e < s1;
+                        const bool above = v && (k[e] >> 20) > b1;
+                        const bool cand = v && (k[e] >> 20) == b1;
+                        eqm |= (unsigned)(cand && k[e] == tau) << e;
+                        selm |= (unsigned)(above || (cand && k[e] > tau)) << e;
+                    }
                 }
+                int eq_tot;
+                int er = eq_before + warp_excl(__popc(eqm), eq_tot);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if ((eqm >> e) & 1u) { selm |= (unsigned)(er < krem) << e; ++er; }
+                int sel_tot;
+                int rank = sel_before + warp_excl(__popc(selm), sel_tot);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if ((selm >> e) & 1u) {
+                        if (rank >= lo && rank < hi) mypos[rank - lo] = base + e;
+                        ++rank;
+                    }
+                eq_before += eq_tot;
+                sel_before += sel_tot;
+                if (sel_before >= hi) break;  // warp-uniform
             }
+            (void)lt_all;
         }
     }
-    const int n_gst = (my_cnt + kGKeys - 1) / kGKeys;
-    auto issue_stage = [&](int st) {
-        // warp 0: lane j copies the K and V rows of the stage's key j
-        if (warp == 0) {
-            const int buf = st % kGStages;
-            uint8_t* kb = region_a + buf * stage_bytes;
-            uint8_t* vb = kb + kGKeys * krow;
-            if (lane == 0) ptx::mbar_arrive_expect_tx(&gath_bar[buf], kGKeys * 2 * P.rowbytes);
-            __syncwarp();
-            int j = st * kGKeys + lane;
-            if (j >= my_cnt) j = st * kGKeys;  // pad with a valid row; masked below
-            const int pos = mypos[j];
-            const bf16* ks;
-            const bf16* vs;
-            if (pos == p) {
-                ks = P.k_new + (int64_t)b * P.H_kv * kD;
-                vs = P.v_new + (int64_t)b * P.H_kv * kD;
-            } else {
-                ks = P.k_cache + ((int64_t)b * P.N_max + pos) * P.H_kv * kD;
-                vs = P.v_cache + ((int64_t)b * P.N_max + pos) * P.H_kv * kD;
-            }
-            ptx::bulk_load(kb + lane * krow, ks, P.rowbytes, &gath_bar[buf]);
-            ptx::bulk_load(vb + lane * krow, vs, P.rowbytes, &gath_bar[buf]);
+    __syncthreads();
+    if (P.idx) {
+        for (int i = tid; i < mine; i += kAttThreads) P.idx[(int64_t)b * P.M + lo + i] = mypos[i];
+        if (j == 0)
+            for (int i = cnt + tid; i < P.M; i += kAttThreads) P.idx[(int64_t)b * P.M + i] = -1;
+    }
+    if (P.count && j == 0 && tid == 0) P.count[b] = cnt;
+
+    // ---- gather + attention over this CTA's positions
+    const int g_w = warp / A::wph, part = warp % A::wph;
+    const int nst = (mine + kGKeys - 1) / kGKeys;
+    constexpr int kb_row = HKV * kD;  // elements per cached row
+
+    uint4 rb[A::chunks_per_thread];  // this thread's 16-byte chunks of one stage
+    auto load_stage = [&](int st) {
+#pragma unroll
+        for (int u = 0; u < A::chunks_per_thread; ++u) {
+            const int c = tid + u * kAttThreads;
+            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
+            const int which = w2 / A::rpc, off = w2 % A::rpc;
+            int jj = st * kGKeys + kk;
+            if (jj >= mine) jj = st * kGKeys;  // pad with a valid row; masked in the softmax
+            const int pos = mypos[jj];
+            const bf16* src = (pos == p)
+                                  ? (which ? P.v_new : P.k_new) + (int64_t)b * kb_row
+                                  : (which ? P.v_cache : P.k_cache) + ((int64_t)b * P.N_max + pos) * kb_row;
+            rb[u] = __ldg(reinterpret_cast<const uint4*>(src) + off);
         }
     };
-    if (ok)
-        for (int st = 0; st < min(n_gst, kGStages); ++st) issue_stage(st);
+    auto store_stage = [&](int st) {
+        uint8_t* dst = stage + (st & 1) * A::stage_bytes;
+#pragma unroll
+        for (int u = 0; u < A::chunks_per_thread; ++u) {
+            const int c = tid + u * kAttThreads;
+            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
+            const int which = w2 / A::rpc, off = w2 % A::rpc;
+            *reinterpret_cast<uint4*>(dst + which * kGKeys * A::krow + kk * A::krow + off * 16) = rb[u];
+        }
+    };
 
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.0f, 0.0f};
-    float oacc[8][4];  // up to 8 n-tiles of 8 dims (dw <= 64)
+    float oacc[A::ntile_o][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int t = 0; t < A::ntile_o; ++t)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[j][e] = 0.0f;
-    const int ntile_o = dw / 8;
+        for (int e = 0; e < 4; ++e) oacc[t][e] = 0.0f;
+    const uint32_t q_base = ptx::smem_u32(qs + g_w * 16 * kQRow);
+    const uint32_t head_off = (uint32_t)(g_w * kD * 2);
 
-    for (int st = 0; st < n_gst; ++st) {
-        const int buf = st % kGStages;
-        const uint32_t parity = (st / kGStages) & 1;
-        if (ok && !ptx::mbar_wait_bounded(&gath_bar[buf], parity, kWaitTries)) {
-            ok = false;
-            if (tid == 0) record_error(P.status, kDevTimeout);
-        }
-        if (ok) {
-            const uint32_t kb = ptx::smem_u32(region_a + buf * stage_bytes);
-            const uint32_t vb = kb + kGKeys * krow;
-            const uint32_t head_off = (uint32_t)(g_w * kD * 2);
-            // S = Q K^T for 32 keys: 4 n-tiles of 8 keys
-            float sc[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sc[nt][e] = 0.0f;
-#pragma unroll
-                for (int ks = 0; ks < 8; ks += 2) {
-                    uint32_t kr[4];
-                    const int key = nt * 8 + (lane & 7);
-                    const int dim0 = ks * 16 + (lane >> 3) * 8;
-                    ptx::ldmatrix_x4(kr, kb + key * krow + head_off + dim0 * 2);
-                    ptx::mma_bf16(sc[nt], qa[ks], kr[0], kr[1]);
-                    ptx::mma_bf16(sc[nt], qa[ks + 1], kr[2], kr[3]);
-                }
-            }
-            // scale, mask, online softmax (rows gid and gid + 8)
-            float mt[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = st * kGKeys + nt * 8 + 2 * tq + (e & 1);
-                    float v = sc[nt][e] * P.scale_log2;
-                    if (key >= my_cnt) v = -INFINITY;
-                    sc[nt][e] = v;
-                    mt[e >> 1] = fmaxf(mt[e >> 1], v);
-                }
-            }
-            float corr[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 1));
-                mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 2));
-                const float m_new = fmaxf(m_run[h], mt[h]);
-                corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m_run[h] - m_new);
-                m_run[h] = m_new;
-                l_run[h] *= corr[h];
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                oacc[j][0] *= corr[0]; oacc[j][1] *= corr[0];
-                oacc[j][2] *= corr[1]; oacc[j][3] *= corr[1];
-            }
-            uint32_t pa[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                float pv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float m = m_run[e >> 1];
-                    pv[e] = (m == -INFINITY) ? 0.0f : exp2f(sc[nt][e] - m);
-                    l_run[e >> 1] += pv[e];
-                }
-                // A fragment of P for k-step nt/2: n-tile 2k -> regs 0,1; 2k+1 -> regs 2,3
-                const int kk = nt >> 1, hi = nt & 1;
-                pa[kk][0 + 2 * hi] = ptx::pack_bf16(pv[0], pv[1]);
-                pa[kk][1 + 2 * hi] = ptx::pack_bf16(pv[2], pv[3]);
-            }
-            // O += P V over this warp's dims
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    if (j < ntile_o) {
-                        uint32_t vr[4];
-                        const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                        const int dim0 = part * dw + (j + (lane >> 4)) * 8;
-                        ptx::ldmatrix_x4_trans(vr, vb + key * krow + head_off + dim0 * 2);
-                        ptx::mma_bf16(oacc[j], pa[kk], vr[0], vr[1]);
-                        ptx::mma_bf16(oacc[j + 1], pa[kk], vr[2], vr[3]);
-                    }
-                }
-            }
-        }
-        __syncthreads();  // buffer free
-        if (ok && st + kGStages < n_gst) issue_stage(st + kGStages);
+    __syncthreads();  // the stage area no longer holds score keys
+    if (nst > 0) {
+        load_stage(0);
+        store_stage(0);
     }
-    // reduce the row sums across the quad
+    __syncthreads();
+#pragma unroll 1
+    for (int st = 0; st < nst; ++st) {
+        if (st + 1 < nst) load_stage(st + 1);  // in flight while this stage computes
+        const uint32_t kb = ptx::smem_u32(stage + (st & 1) * A::stage_bytes);
+        const uint32_t vb = kb + kGKeys * A::krow;
+        float sc[4][4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[t][e] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ks += 2) {
+            uint32_t qa0[4], qa1[4];
+            {
+                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int col = ks * 16 + (lane >> 4) * 8;
+                ptx::ldmatrix_x4(qa0, q_base + row * kQRow + col * 2);
+                ptx::ldmatrix_x4(qa1, q_base + row * kQRow + (col + 16) * 2);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                uint32_t kr[4];
+                const int key = nt * 8 + (lane & 7);
+                const int dim0 = ks * 16 + (lane >> 3) * 8;
+                ptx::ldmatrix_x4(kr, kb + key * A::krow + head_off + dim0 * 2);
+                ptx::mma_bf16(sc[nt], qa0, kr[0], kr[1]);
+                ptx::mma_bf16(sc[nt], qa1, kr[2], kr[3]);
+            }
+        }
+        float mt[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = st * kGKeys + nt * 8 + 2 * tq + (e & 1);
+                float v = sc[nt][e] * P.scale_log2;
+                if (key >= mine) v = -INFINITY;
+                sc[nt][e] = v;
+                mt[e >> 1] = fmaxf(mt[e >> 1], v);
+            }
+        float corr[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 1));
+            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 2));
+            const float m_new = fmaxf(m_run[h], mt[h]);
+            corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m_run[h] - m_new);
+            m_run[h] = m_new;
+            l_run[h] *= corr[h];
+        }
+#pragma unroll
+        for (int t = 0; t < A::ntile_o; ++t) {
+            oacc[t][0] *= corr[0]; oacc[t][1] *= corr[0];
+            oacc[t][2] *= corr[1]; oacc[t][3] *= corr[1];
+        }
+        uint32_t pa[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float m = m_run[e >> 1];
+                pv[e] = (m == -INFINITY) ? 0.0f : exp2f(sc[nt][e] - m);
+                l_run[e >> 1] += pv[e];
+            }
+            const int kk = nt >> 1, hi2 = nt & 1;
+            pa[kk][0 + 2 * hi2] = ptx::pack_bf16(pv[0], pv[1]);
+            pa[kk][1 + 2 * hi2] = ptx::pack_bf16(pv[2], pv[3]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+            for (int t = 0; t < A::ntile_o; t += 2) {
+                uint32_t vr[4];
+                const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+                const int dim0 = part * A::dw + (t + (lane >> 4)) * 8;
+                ptx::ldmatrix_x4_trans(vr, vb + key * A::krow + head_off + dim0 * 2);
+                ptx::mma_bf16(oacc[t], pa[kk], vr[0], vr[1]);
+                ptx::mma_bf16(oacc[t + 1], pa[kk], vr[2], vr[3]);
+            }
+        }
+        if (st + 1 < nst) store_stage(st + 1);
+        __syncthreads();
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
         l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
     }
-    // partials into region A: m, l per (g, row); O per (g, row, dim)
-    __syncthreads();
-    float* part_m = reinterpret_cast<float*>(region_a);
-    float* part_l = part_m + P.H_kv * 16;
-    float* part_o = part_l + P.H_kv * 16;
-    {
+    // partial (m, l, O) of this CTA for the query heads of group g_w
+    float* prow = P.part + ((int64_t)b * P.S2 + j) * P.H_q * (kD + 2);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int row = gid + 8 * h;
+    for (int h = 0; h < 2; ++h) {
+        const int row = gid + 8 * h;
+        if (row < P.group) {
+            float* rec = prow + (int64_t)(g_w * P.group + row) * (kD + 2);
             if (part == 0 && tq == 0) {
-                part_m[g_w * 16 + row] = m_run[h];
-                part_l[g_w * 16 + row] = l_run[h];
+                rec[0] = m_run[h];
+                rec[1] = l_run[h];
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (j < ntile_o) {
-                    const int dim = part * dw + j * 8 + 2 * tq;
-                    float* dst = part_o + (g_w * 16 + row) * kD + dim;
-                    dst[0] = oacc[j][2 * h];
-                    dst[1] = oacc[j][2 * h + 1];
-                }
+            for (int t = 0; t < A::ntile_o; ++t) {
+                const int dim = part * A::dw + t * 8 + 2 * tq;
+                rec[2 + dim] = oacc[t][2 * h];
+                rec[2 + dim + 1] = oacc[t][2 * h + 1];
             }
         }
     }
-    ptx::cluster_sync();  // partials visible cluster-wide
 
-    // ---------------------------------------------------------------- D: combine + gate
-    for (int e = tid; e < P.group * P.ncols; e += kThreads) {
-        const int h = e / P.ncols, c = e % P.ncols;
-        const int prow = g_r * 16 + h;
-        float mx = -INFINITY;
-        float mc[16], lc[16];
-        for (int cc = 0; cc < C; ++cc) {
-            mc[cc] = ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_u32(part_m + prow), cc));
-            lc[cc] = ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_u32(part_l + prow), cc));
-            mx = fmaxf(mx, mc[cc]);
+}
+
+// ============================================================================ K3: combine
+// One CTA per (sequence, query head), one thread per output dimension: merge
+// the attend CTAs' partial (max, sum, output) triples, mix with the linear
+// branch through the gate, write o.  Also advances the elu+1 normaliser z and
+// clears the sequence's key histogram for the next call.
+__global__ void __launch_bounds__(kD) k_decode_combine(const Params P) {
+    const int b = blockIdx.x / P.H_q, h = blockIdx.x % P.H_q, c = threadIdx.x;
+    ptx::pdl_wait_prior();  // the attend kernel's partials are complete
+    const int64_t jstride = (int64_t)P.H_q * (kD + 2);
+    const float* rec0 = P.part + ((int64_t)b * P.S2 * P.H_q + h) * (kD + 2);
+    float M = -INFINITY, Lsum = 0.0f, O = 0.0f;
+#pragma unroll 1
+    for (int j0 = 0; j0 < P.S2; j0 += 8) {
+        float mm[8], ll[8], oo[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            mm[u] = -INFINITY;
+            ll[u] = 0.0f;
+            oo[u] = 0.0f;
+            if (j0 + u < P.S2) {
+                const float* rec = rec0 + (j0 + u) * jstride;
+                mm[u] = __ldg(rec);
+                ll[u] = __ldg(rec + 1);
+                oo[u] = __ldg(rec + 2 + c);
+            }
         }
-        float num = 0.0f, dsum = 0.0f;
-        for (int cc = 0; cc < C; ++cc) {
-            if (mc[cc] == -INFINITY) continue;
-            const float f = exp2f(mc[cc] - mx);
-            dsum = fmaf(lc[cc], f, dsum);
-            num = fmaf(ptx::ld_dsmem_f32(ptx::mapa(ptx::smem_u32(part_o + prow * kD + c0 + c), cc)),
-                       f, num);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (mm[u] == -INFINITY) continue;
+            const float nm = fmaxf(M, mm[u]);
+            const float a = exp2f(M - nm), w = exp2f(mm[u] - nm);
+            Lsum = fmaf(Lsum, a, ll[u] * w);
+            O = fmaf(O, a, oo[u] * w);
+            M = nm;
         }
-        const float o_sp = dsum > 0.0f ? num / dsum : 0.0f;
-        const int hq = g_r * P.group + h;
-        const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + hq]);
-        const float g = 1.0f / (1.0f + __expf(-x));
-        const float out = g * olin[h * P.ncols + c] + (1.0f - g) * o_sp;
-        P.o[((int64_t)b * P.H_q + hq) * kD + c0 + c] = __float2bfloat16_rn(out);
     }
-    ptx::cluster_sync();  // nobody exits while others still read its shared memory
-    if (!ok && tid == 0) {
-        // A bounded wait gave up: give the copies still in flight another bounded
-        // chance to land before the shared memory they target is released.
-        for (int i = 0; i < kScanStages + kGStages; ++i)
-            for (uint32_t par = 0; par < 2; ++par) ptx::mbar_wait_bounded(&bars[i], par, 1u << 16);
+    const float o_sp = Lsum > 0.0f ? O / Lsum : 0.0f;
+    const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + h]);
+    const float gt = 1.0f / (1.0f + __expf(-x));
+    const float o_lin = __ldg(P.olin + ((int64_t)b * P.H_q + h) * kD + c);
+    P.o[((int64_t)b * P.H_q + h) * kD + c] = __float2bfloat16_rn(gt * o_lin + (1.0f - gt) * o_sp);
+    if (P.phi == LISA_PHI_ELU1_NORM && h < P.H_kv) {
+        // z <- z + phi(k_L): every reader of the old z (the scan kernel) has finished
+        const int64_t zi = ((int64_t)b * P.H_kv + h) * kD + c;
+        P.z[zi] += feat(P.phi, __bfloat162float(P.k_L[zi]));
+    }
+    if (h == 0) {
+        uint4* hz = reinterpret_cast<uint4*>(P.hist + (int64_t)b * 4096);
+        for (int i = c; i < 4096 / 4; i += kD) hz[i] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
-// ---------------------------------------------------------------- host side
+// ============================================================================ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -771,53 +931,63 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-int pick_cluster(const Shape& s) {
-    // 16 CTAs per sequence when the GPU can hold such clusters and there is
-    // not already enough work to fill it with clusters of 8.
-    static int can16 = -1;
-    if (can16 < 0) {
-        can16 = 0;
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 16;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(16);
-        cfg.blockDim = dim3(kThreads);
-        const Smem L = smem_plan(16, kMaxKPC, 64, 1024, 4);
-        cfg.dynamicSmemBytes = L.total;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        auto kern = k_decode_fused<16>;
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess && nclusters >= 1)
-            can16 = 1;
-        cudaGetLastError();
+int num_sms() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
     }
-    if (!can16) return 8;
-    return s.B * 8 >= 2 * 148 ? 8 : 16;
+    return sms;
+}
+
+struct Plan {
+    int S1, KPC, S2, per, ns;
+    size_t scores, olin, part, hist, end;
+};
+
+Plan make_plan(const Shape& s) {
+    Plan pl;
+    const int sms = num_sms();
+    const int n = s.L;
+    pl.S1 = std::max(1, std::min(sms / std::max(1, s.B), (n + 15) / 16));
+    pl.KPC = align_up((n + pl.S1 - 1) / pl.S1, 16);
+    pl.S1 = (n + pl.KPC - 1) / pl.KPC;
+    const int cnt = std::min(s.M, n);
+    pl.S2 = std::max(1, std::min(sms / std::max(1, s.B), (cnt + 31) / 32));
+    pl.per = (cnt + pl.S2 - 1) / pl.S2;
+    pl.S2 = (cnt + pl.per - 1) / pl.per;
+    pl.ns = align_up(n, 32);
+    size_t off = kStatusBytes;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return at;
+    };
+    pl.scores = take(sizeof(float) * (size_t)s.B * pl.ns);
+    pl.olin = take(sizeof(float) * (size_t)s.B * s.H_q * kD);
+    pl.part = take(sizeof(float) * (size_t)s.B * pl.S2 * s.H_q * (kD + 2));
+    pl.hist = take(sizeof(unsigned) * (size_t)s.B * 4096);
+    pl.end = off;
+    return pl;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
 
-size_t fast_decode_ws_bytes(const Shape&) { return kStatusBytes; }
+size_t fast_decode_ws_bytes(const Shape& s) {
+    if (s.B <= 0 || s.L <= 0) return kStatusBytes;
+    return make_plan(s).end;
+}
 
 bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
     if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD || s.d_I != kDI || s.H_Ik != 1) return false;
     if (s.H_I > 8 || s.group > 16 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
-    if (s.L < 1 || s.M < 1) return false;
-    const int C = pick_cluster(s);
-    const int KPC = align_up((s.L + C - 1) / C, 16);
-    if (KPC > kMaxKPC) return false;
-    const int cnt = s.M < s.L ? s.M : s.L;
-    if ((cnt + C - 1) / C > kMaxPer) return false;
-    const Smem L = smem_plan(C, KPC, s.H_kv * kD / C, s.H_kv * kD * 2, s.H_kv);
-    if (L.total > 227 * 1024) return false;
+    if (s.L < 1 || s.M < 1 || s.B < 1) return false;
+    const Plan pl = make_plan(s);
+    if (pl.per > kMaxPer) return false;
     const void* ptrs[] = {a.q, a.k_new, a.v_new, a.q_I, a.k_I_new, a.q_L, a.k_L, a.v_L,
                           a.k_cache, a.v_cache, a.k_I_cache, a.S, a.o};
     for (const void* p : ptrs)
@@ -827,13 +997,13 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
     return true;
 }
 
-template <int C>
-cudaError_t launch_decode(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st) {
+cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st) {
+    const Plan pl = make_plan(s);
     Params P;
-    P.B = s.B; P.n = s.L; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv; P.group = s.group;
-    P.H_I = s.H_I; P.M = s.M; P.phi = s.phi;
-    P.KPC = align_up((s.L + C - 1) / C, 16);
-    P.ncols = s.H_kv * kD / C;
+    P.B = s.B; P.n = s.L; P.ns = pl.ns; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv;
+    P.group = s.group; P.H_I = s.H_I; P.M = s.M; P.phi = s.phi;
+    P.S1 = pl.S1; P.KPC = pl.KPC; P.S2 = pl.S2; P.per = pl.per;
+    P.la_slices = s.B * s.H_kv * (kD / kLaCols);
     P.rowbytes = s.H_kv * kD * 2;
     P.scale_log2 = s.sm_scale * 1.4426950408889634f;
     P.q = (const bf16*)a.q; P.k_new = (const bf16*)a.k_new; P.v_new = (const bf16*)a.v_new;
@@ -842,7 +1012,12 @@ cudaError_t launch_decode(const Shape& s, const lisa_decode_args& a, void* ws, c
     P.gate = (const bf16*)a.gate_logit_lin;
     P.k_cache = (bf16*)a.k_cache; P.v_cache = (bf16*)a.v_cache; P.k_I_cache = (bf16*)a.k_I_cache;
     P.S = a.S; P.z = a.z; P.o = (bf16*)a.o; P.idx = a.idx; P.count = a.count;
+    char* w8 = (char*)ws;
     P.status = (unsigned*)ws;
+    P.scores = (float*)(w8 + pl.scores);
+    P.olin = (float*)(w8 + pl.olin);
+    P.part = (float*)(w8 + pl.part);
+    P.hist = (unsigned*)(w8 + pl.hist);
 
     CUtensorMap tmap;
     const cuuint64_t gdim[2] = {(cuuint64_t)kDI, (cuuint64_t)s.B * (cuuint64_t)s.N_max};
@@ -855,33 +1030,47 @@ cudaError_t launch_decode(const Shape& s, const lisa_decode_args& a, void* ws, c
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    const Smem L = smem_plan(C, P.KPC, P.ncols, P.rowbytes, P.H_kv);
-    auto kern = k_decode_fused<C>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
-    if (e != cudaSuccess) return e;
-    if (C > 8) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    static bool attrs_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attrs_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_decode_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             ScanSmem::total);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_decode_attend<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Att<1>::total);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_decode_attend<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Att<2>::total);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_decode_attend<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Att<4>::total);
         if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attrs_set[dev] = true;
     }
+    k_decode_scan<<<s.B * pl.S1, kScanThreads + kLaThreads, ScanSmem::total, st>>>(tmap, P);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(s.B * C);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = L.total;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(s.B * pl.S2);
+    cfg.blockDim = dim3(kAttThreads);
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, tmap, P);
-}
-
-cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st) {
-    const int C = pick_cluster(s);
-    if (C == 16) return launch_decode<16>(s, a, ws, st);
-    return launch_decode<8>(s, a, ws, st);
+    switch (s.H_kv) {
+        case 1: cfg.dynamicSmemBytes = Att<1>::total; e = cudaLaunchKernelEx(&cfg, k_decode_attend<1>, P); break;
+        case 2: cfg.dynamicSmemBytes = Att<2>::total; e = cudaLaunchKernelEx(&cfg, k_decode_attend<2>, P); break;
+        default: cfg.dynamicSmemBytes = Att<4>::total; e = cudaLaunchKernelEx(&cfg, k_decode_attend<4>, P); break;
+    }
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(s.B * s.H_q);
+    cfg.blockDim = dim3(kD);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, k_decode_combine, P);
 }
 
 }  // namespace lisa
