@@ -302,17 +302,18 @@ def run_gpu(args, wl, rank, world, device):
                          f"(caches, state, inputs) used in rotation, "
                          f"{args.rotate} x {bytes_['total'] / 1e6:.1f} MB touched per cycle",
                    "step": "decode step: append, linear update+readout, indexer scan, "
-                           "top-M, sparse attention, gate (2 kernels, PDL-chained)"},
+                           "top-M, sparse attention, gate (3 kernels, PDL-chained)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "frac_of_8TBs": achieved / 8000.0,
                      "traffic": _profiled_traffic(wl),
                      "algorithmic_bytes_per_launch": bytes_["total"],
-                     "kernel": "decode step (k_decode_scan + k_decode_attend)",
+                     "kernel": "decode step: one lisa_decode_step call = k_decode_scan + "
+                               "k_decode_attend + k_decode_combine (PDL-chained)",
                      "launch_us": avg_s * 1e6},
         "e2e": {"value": world * B * args.steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
         "step_ms_min": min(times_ms), "step_ms_median": statistics.median(times_ms),
     }
