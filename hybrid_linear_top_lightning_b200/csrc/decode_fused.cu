@@ -40,7 +40,9 @@
 
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
+#include "select_row.cuh"
 #include "sm100_ptx.cuh"
+#include "tma_host.cuh"
 
 namespace lisa {
 namespace {
@@ -59,7 +61,6 @@ constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kGKeys = 32;            // keys per gather stage
 constexpr int kMaxPer = 2048;         // selected positions per attend CTA
 constexpr int kQRow = kD * 2 + 16;    // padded shared-memory row of a query (bytes)
-constexpr int kCandCap = 256;         // threshold-bin candidates per warp (more: full passes)
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
@@ -403,28 +404,6 @@ struct Att {
     static constexpr int key_cap = 2 * stage_bytes / 4 - 32;  // scores that fit in the stages
 };
 
-__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    int off = 0;
-    total = 0;
-#pragma unroll
-    for (int w = 0; w < kAttWarps; ++w) {
-        const int x = scratch[w];
-        if (w < warp) off += x;
-        total += x;
-    }
-    __syncthreads();
-    return off + incl - v;
-}
-
 template <int HKV>
 __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P) {
     using A = Att<HKV>;
@@ -432,7 +411,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     unsigned* hist = reinterpret_cast<unsigned*>(att_raw + A::hist);
     uint64_t* rowbar = reinterpret_cast<uint64_t*>(att_raw + A::bar);
     int* bc = reinterpret_cast<int*>(att_raw + A::bc);
-    int* scratch = bc + 32;
     int* mypos = reinterpret_cast<int*>(att_raw + A::mypos);
     uint8_t* qs = att_raw + A::q;
     uint8_t* stage = att_raw + A::stage;
@@ -470,226 +448,21 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     if (n <= P.M) {
         for (int i = tid; i < mine; i += kAttThreads) mypos[i] = lo + i;
     } else {
-        float* srow_s = reinterpret_cast<float*>(stage);
+        // the score row comes into shared memory by TMA bulk copies when it fits
         const bool resident = n <= A::key_cap;
-        bool row_ok = true;
         if (resident && tid == 0) {
             const int bytes = ((n + 3) / 4) * 16;
             ptx::mbar_arrive_expect_tx(rowbar, bytes);
             for (int off = 0; off < bytes; off += 16384)
                 ptx::bulk_load(stage + off, srow + off / 4, min(16384, bytes - off), rowbar);
         }
-        // first digit from the sequence histogram (while the row is in flight)
-        auto find_bin = [&](const unsigned* hv, int bpt, int tsum, int need) {
-            int total;
-            const int below = block_excl_scan(tsum, scratch, total);
-            const int above = total - below - tsum;
-            if (tid == 0) { bc[0] = 0; bc[1] = 1; }
-            __syncthreads();
-            if (above < need && need <= above + tsum) {
-                int acc = above;
-                for (int q = bpt - 1; q >= 0; --q) {
-                    if (acc + (int)hv[q] >= need) {
-                        bc[0] = tid * bpt + q;
-                        bc[1] = need - acc;
-                        break;
-                    }
-                    acc += (int)hv[q];
-                }
-            }
-            __syncthreads();
-        };
-        uint32_t b1;
-        int krem;
-        {
-            unsigned hv[16];
-            int tsum = 0;
-            const uint4* g4 = reinterpret_cast<const uint4*>(P.hist + (int64_t)b * 4096) + tid * 4;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 u = __ldcg(g4 + q);
-                hv[4 * q] = u.x; hv[4 * q + 1] = u.y; hv[4 * q + 2] = u.z; hv[4 * q + 3] = u.w;
-            }
-#pragma unroll
-            for (int q = 0; q < 16; ++q) tsum += (int)hv[q];
-            find_bin(hv, 16, tsum, P.M);
-            b1 = (uint32_t)bc[0];
-            krem = bc[1];
-        }
-        if (resident && !ptx::mbar_wait_bounded(rowbar, 0, kWaitTries)) {
-            row_ok = false;
-            if (tid == 0) record_error(P.status, kDevTimeout);
-        }
-        const float* rsrc = resident ? srow_s : srow;
-        auto keys8 = [&](int base, uint32_t (&k)[8]) {
-            const float4* src = reinterpret_cast<const float4*>(rsrc) + base / 4;
-            float4 v0, v1;
-            if (resident) { v0 = src[0]; v1 = src[1]; }
-            else { v0 = __ldcg(src); v1 = __ldcg(src + 1); }
-            k[0] = order_key(v0.x); k[1] = order_key(v0.y); k[2] = order_key(v0.z); k[3] = order_key(v0.w);
-            k[4] = order_key(v1.x); k[5] = order_key(v1.y); k[6] = order_key(v1.z); k[7] = order_key(v1.w);
-        };
-        auto warp_excl = [&](int v, int& tot) {
-            int incl = v;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            tot = __shfl_sync(0xffffffffu, incl, 31);
-            return incl - v;
-        };
-        // Warp w owns positions [w*seg, (w+1)*seg), walked in blocks of 256 with
-        // lane l on the 8 consecutive positions blk + 8l .. blk + 8l + 7.
-        const int seg = ((n + kAttWarps - 1) / kAttWarps + 255) / 256 * 256;
-        const int s0 = warp * seg, s1 = min(n, s0 + seg);
-        uint2* clist = reinterpret_cast<uint2*>(att_raw + A::cand) + warp * kCandCap;
-        // scan A: keys above the first digit, and the threshold-digit candidates (in order)
-        int n_above = 0, ncand = 0;
-        if (row_ok) {
-#pragma unroll 1
-            for (int blk = s0; blk < s1; blk += 256) {
-                const int base = blk + lane * 8;
-                uint32_t k[8];
-                unsigned cm = 0;
-                if (base < s1) {
-                    keys8(base, k);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const bool v = base + e < s1;
-                        n_above += v && (k[e] >> 20) > b1;
-                        cm |= (unsigned)(v && (k[e] >> 20) == b1) << e;
-                    }
-                }
-                int ctot;
-                int w = ncand + warp_excl(__popc(cm), ctot);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if ((cm >> e) & 1u) {
-                        if (w < kCandCap) clist[w] = make_uint2(k[e], (uint32_t)(base + e));
-                        ++w;
-                    }
-                ncand += ctot;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
-        if (lane == 0) { scratch[8 + warp] = n_above; scratch[16 + warp] = ncand; }
-        __syncthreads();
-        bool overflow = false;
-        for (int w = 0; w < kAttWarps; ++w) overflow |= scratch[16 + w] > kCandCap;
-        // refine: 10 bits, then 10 bits, over the candidates (or, if a warp's
-        // list overflowed, over every key of the row with the first digit b1)
-        uint32_t prefix = b1 << 20, mask = 0xFFFu << 20;
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 10 : 0;
-            for (int i = tid; i < 1024; i += kAttThreads) hist[i] = 0u;
-            __syncthreads();
-            if (row_ok) {
-                if (!overflow) {
-                    for (int i = tid; i < kAttWarps * kCandCap; i += kAttThreads) {
-                        const int w = i / kCandCap, c = i % kCandCap;
-                        if (c < scratch[16 + w]) {
-                            const uint32_t k = reinterpret_cast<const uint2*>(att_raw + A::cand)[i].x;
-                            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 1023u], 1u);
-                        }
-                    }
-                } else {
-                    for (int i8 = tid * 8; i8 < n; i8 += kAttThreads * 8) {
-                        uint32_t k[8];
-                        keys8(i8, k);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            if (i8 + e < n && (k[e] & mask) == prefix)
-                                atomicAdd(&hist[(k[e] >> shift) & 1023u], 1u);
-                    }
-                }
-            }
-            __syncthreads();
-            unsigned hv[4];
-            int tsum = 0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) { hv[q] = hist[tid * 4 + q]; tsum += (int)hv[q]; }
-            find_bin(hv, 4, tsum, krem);
-            prefix |= (uint32_t)bc[0] << shift;
-            krem = bc[1];
-            mask |= 1023u << shift;
-            __syncthreads();
-        }
-        const uint32_t tau = prefix;  // the M-th largest key; krem of its ties are kept
-        // selected count of each warp's segment: keys above b1, plus candidates
-        // above tau, plus the ties that fall to it in position order
-        int gt_c = 0, eq_c = 0;
-        if (!overflow) {
-            for (int c = lane; c < scratch[16 + warp]; c += 32) {
-                const uint32_t k = clist[c].x;
-                gt_c += k > tau;
-                eq_c += k == tau;
-            }
-        } else if (row_ok) {
-            for (int blk = s0; blk < s1; blk += 256) {
-                const int base = blk + lane * 8;
-                if (base >= s1) continue;
-                uint32_t k[8];
-                keys8(base, k);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (base + e < s1 && (k[e] >> 20) == b1) { gt_c += k[e] > tau; eq_c += k[e] == tau; }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            gt_c += __shfl_xor_sync(0xffffffffu, gt_c, o);
-            eq_c += __shfl_xor_sync(0xffffffffu, eq_c, o);
-        }
-        if (lane == 0) { scratch[24 + warp] = gt_c; scratch[32 + warp] = eq_c; }
-        __syncthreads();
-        int eq_before = 0, sel_before = 0;
-        for (int w = 0; w < warp; ++w) {
-            const int eqw = scratch[32 + w];
-            sel_before += scratch[8 + w] + scratch[24 + w] + max(0, min(eqw, krem - eq_before));
-            eq_before += eqw;
-        }
-        const int sel_w = n_above + gt_c + max(0, min(eq_c, krem - eq_before));
-        // ranked walk, only where this warp's ranks meet this CTA's share [lo, hi)
-        if (row_ok && sel_before < hi && sel_before + sel_w > lo) {
-            const unsigned lt_all = 0xffffffffu;
-#pragma unroll 1
-            for (int blk = s0; blk < s1; blk += 256) {
-                const int base = blk + lane * 8;
-                uint32_t k[8];
-                unsigned eqm = 0, selm = 0;
-                if (base < s1) {
-                    keys8(base, k);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const bool v = base + e < s1;
-                        const bool above = v && (k[e] >> 20) > b1;
-                        const bool cand = v && (k[e] >> 20) == b1;
-                        eqm |= (unsigned)(cand && k[e] == tau) << e;
-                        selm |= (unsigned)(above || (cand && k[e] > tau)) << e;
-                    }
-                }
-                int eq_tot;
-                int er = eq_before + warp_excl(__popc(eqm), eq_tot);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if ((eqm >> e) & 1u) { selm |= (unsigned)(er < krem) << e; ++er; }
-                int sel_tot;
-                int rank = sel_before + warp_excl(__popc(selm), sel_tot);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if ((selm >> e) & 1u) {
-                        if (rank >= lo && rank < hi) mypos[rank - lo] = base + e;
-                        ++rank;
-                    }
-                eq_before += eq_tot;
-                sel_before += sel_tot;
-                if (sel_before >= hi) break;  // warp-uniform
-            }
-            (void)lt_all;
-        }
+        SelectSmem sel;
+        sel.hist = hist;
+        sel.bc = bc;
+        sel.cand = reinterpret_cast<uint2*>(att_raw + A::cand);
+        row_topm(resident ? reinterpret_cast<const float*>(stage) : srow, resident, n, P.M,
+                 P.hist + (int64_t)b * 4096, sel, lo, hi, mypos, resident ? rowbar : nullptr,
+                 P.status);
     }
     __syncthreads();
     if (P.idx) {
@@ -911,26 +684,6 @@ __global__ void __launch_bounds__(kD) k_decode_combine(const Params P) {
 }
 
 // ============================================================================ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 int num_sms() {
     static int sms = 0;
     if (!sms) {
@@ -993,7 +746,7 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
     for (const void* p : ptrs)
         if (!aligned16(p)) return false;
     if (s.phi == LISA_PHI_ELU1_NORM && !aligned16(a.z)) return false;
-    if (!encode_fn()) return false;
+    if (!tma_encode_fn()) return false;
     return true;
 }
 
@@ -1020,14 +773,7 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     P.hist = (unsigned*)(w8 + pl.hist);
 
     CUtensorMap tmap;
-    const cuuint64_t gdim[2] = {(cuuint64_t)kDI, (cuuint64_t)s.B * (cuuint64_t)s.N_max};
-    const cuuint64_t gstride[1] = {(cuuint64_t)kDI * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kDI, (cuuint32_t)kScanRows};
-    const cuuint32_t estride[2] = {1, 1};
-    if (encode_fn()(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.k_I_cache, gdim, gstride, box,
-                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max, kScanRows))
         return cudaErrorInvalidValue;
 
     static bool attrs_set[64] = {};

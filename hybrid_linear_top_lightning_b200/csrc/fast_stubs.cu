@@ -3,10 +3,6 @@
 
 namespace lisa {
 
-size_t fast_topm_ws_bytes(const Shape&) { return 0; }
-bool fast_topm_supported(const Shape&, const void*, const void*, const float*, int64_t) { return false; }
-cudaError_t fast_topm(const Shape&, const void*, const void*, const float*, int64_t, int32_t*,
-                      int32_t*, void*, cudaStream_t) { return cudaErrorNotSupported; }
 
 size_t fast_attention_ws_bytes(const Shape&, bool) { return 0; }
 bool fast_attention_supported(const Shape&, const void*, const void*, const void*, bool) { return false; }
