@@ -40,6 +40,7 @@
 
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
+#include "attend_core.cuh"
 #include "select_row.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
@@ -56,11 +57,7 @@ constexpr int kScanRows = 128;        // keys per TMA box (16 per warp)
 constexpr int kScanStages = 8;        // boxes in flight per CTA
 constexpr int kBoxBytes = kScanRows * kDI * 2;
 constexpr int kLaCols = 32;           // linear-state columns per slice
-constexpr int kAttThreads = 256;
-constexpr int kAttWarps = kAttThreads / 32;
-constexpr int kGKeys = 32;            // keys per gather stage
 constexpr int kMaxPer = 2048;         // selected positions per attend CTA
-constexpr int kQRow = kD * 2 + 16;    // padded shared-memory row of a query (bytes)
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
@@ -383,25 +380,19 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
 
 // ============================================================================ K2: attend
 template <int HKV>
-struct Att {
-    static constexpr int rowbytes = HKV * kD * 2;     // one cached K (or V) row
-    static constexpr int krow = rowbytes + 16;        // padded shared-memory row
-    static constexpr int rpc = rowbytes / 16;         // 16-byte chunks per row
-    static constexpr int stage_bytes = kGKeys * 2 * krow;
-    static constexpr int chunks_per_thread = kGKeys * 2 * rpc / kAttThreads;
-    static constexpr int wph = kAttWarps / HKV;       // warps per KV head
-    static constexpr int dw = kD / wph;               // output dims per warp
-    static constexpr int ntile_o = dw / 8;
-    // shared memory: histogram, broadcasts, selected positions, queries, stages
-    static constexpr int hist = 0;                     // two 2048-bin halves (warps 0-3, 4-7)
-    static constexpr int bar = hist + 2 * 2048 * 4;
-    static constexpr int bc = bar + 16;                 // int[128]: broadcasts, scratch
+struct Att : AttGeo<HKV> {
+    using G = AttGeo<HKV>;
+    // shared memory: histogram, barrier, broadcasts, selected positions,
+    // queries, candidate lists, gather stages (the score row during selection)
+    static constexpr int hist = 0;                     // u32[4096]
+    static constexpr int bar = hist + 4096 * 4;
+    static constexpr int bc = bar + 16;                 // int[128]
     static constexpr int mypos = bc + 128 * 4;
     static constexpr int q = mypos + kMaxPer * 4;
-    static constexpr int cand = q + ((HKV * 16 * kQRow + 127) / 128) * 128;  // uint2[8][kCandCap]
+    static constexpr int cand = q + G::qbytes;          // uint2[8][kCandCap]
     static constexpr int stage = cand + kAttWarps * kCandCap * 8;
-    static constexpr int total = stage + 2 * stage_bytes;
-    static constexpr int key_cap = 2 * stage_bytes / 4 - 32;  // scores that fit in the stages
+    static constexpr int total = stage + 2 * G::stage_bytes;
+    static constexpr int key_cap = 2 * G::stage_bytes / 4 - 32;  // scores that fit in the stages
 };
 
 template <int HKV>
@@ -422,13 +413,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     ptx::pdl_launch_dependents();
 
     // ---- prologue (inputs only; nothing written by the scan kernel)
-    for (int e = tid; e < HKV * 16 * (kD / 8); e += kAttThreads) {
-        const int g = e / (16 * (kD / 8)), r = (e / (kD / 8)) % 16, c = e % (kD / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < P.group)
-            v = reinterpret_cast<const uint4*>(P.q + ((int64_t)b * P.H_q + g * P.group + r) * kD)[c];
-        *reinterpret_cast<uint4*>(qs + (g * 16 + r) * kQRow + c * 16) = v;
-    }
+    attn_load_query<HKV>(qs, P.q + (int64_t)b * P.H_q * kD, P.group);
     if (tid == 0) {
         ptx::mbar_init(rowbar, 1);
         ptx::fence_mbar_init();
@@ -474,141 +459,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
 
     // ---- gather + attention over this CTA's positions
     const int g_w = warp / A::wph, part = warp % A::wph;
-    const int nst = (mine + kGKeys - 1) / kGKeys;
-    constexpr int kb_row = HKV * kD;  // elements per cached row
-
-    uint4 rb[A::chunks_per_thread];  // this thread's 16-byte chunks of one stage
-    auto load_stage = [&](int st) {
-#pragma unroll
-        for (int u = 0; u < A::chunks_per_thread; ++u) {
-            const int c = tid + u * kAttThreads;
-            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
-            const int which = w2 / A::rpc, off = w2 % A::rpc;
-            int jj = st * kGKeys + kk;
-            if (jj >= mine) jj = st * kGKeys;  // pad with a valid row; masked in the softmax
-            const int pos = mypos[jj];
-            const bf16* src = (pos == p)
-                                  ? (which ? P.v_new : P.k_new) + (int64_t)b * kb_row
-                                  : (which ? P.v_cache : P.k_cache) + ((int64_t)b * P.N_max + pos) * kb_row;
-            rb[u] = __ldg(reinterpret_cast<const uint4*>(src) + off);
-        }
-    };
-    auto store_stage = [&](int st) {
-        uint8_t* dst = stage + (st & 1) * A::stage_bytes;
-#pragma unroll
-        for (int u = 0; u < A::chunks_per_thread; ++u) {
-            const int c = tid + u * kAttThreads;
-            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
-            const int which = w2 / A::rpc, off = w2 % A::rpc;
-            *reinterpret_cast<uint4*>(dst + which * kGKeys * A::krow + kk * A::krow + off * 16) = rb[u];
-        }
-    };
-
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.0f, 0.0f};
-    float oacc[A::ntile_o][4];
-#pragma unroll
-    for (int t = 0; t < A::ntile_o; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[t][e] = 0.0f;
-    const uint32_t q_base = ptx::smem_u32(qs + g_w * 16 * kQRow);
-    const uint32_t head_off = (uint32_t)(g_w * kD * 2);
-
-    __syncthreads();  // the stage area no longer holds score keys
-    if (nst > 0) {
-        load_stage(0);
-        store_stage(0);
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int st = 0; st < nst; ++st) {
-        if (st + 1 < nst) load_stage(st + 1);  // in flight while this stage computes
-        const uint32_t kb = ptx::smem_u32(stage + (st & 1) * A::stage_bytes);
-        const uint32_t vb = kb + kGKeys * A::krow;
-        float sc[4][4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[t][e] = 0.0f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ks += 2) {
-            uint32_t qa0[4], qa1[4];
-            {
-                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int col = ks * 16 + (lane >> 4) * 8;
-                ptx::ldmatrix_x4(qa0, q_base + row * kQRow + col * 2);
-                ptx::ldmatrix_x4(qa1, q_base + row * kQRow + (col + 16) * 2);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                uint32_t kr[4];
-                const int key = nt * 8 + (lane & 7);
-                const int dim0 = ks * 16 + (lane >> 3) * 8;
-                ptx::ldmatrix_x4(kr, kb + key * A::krow + head_off + dim0 * 2);
-                ptx::mma_bf16(sc[nt], qa0, kr[0], kr[1]);
-                ptx::mma_bf16(sc[nt], qa1, kr[2], kr[3]);
-            }
-        }
-        float mt[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = st * kGKeys + nt * 8 + 2 * tq + (e & 1);
-                float v = sc[nt][e] * P.scale_log2;
-                if (key >= mine) v = -INFINITY;
-                sc[nt][e] = v;
-                mt[e >> 1] = fmaxf(mt[e >> 1], v);
-            }
-        float corr[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 1));
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 2));
-            const float m_new = fmaxf(m_run[h], mt[h]);
-            corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m_run[h] - m_new);
-            m_run[h] = m_new;
-            l_run[h] *= corr[h];
-        }
-#pragma unroll
-        for (int t = 0; t < A::ntile_o; ++t) {
-            oacc[t][0] *= corr[0]; oacc[t][1] *= corr[0];
-            oacc[t][2] *= corr[1]; oacc[t][3] *= corr[1];
-        }
-        uint32_t pa[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            float pv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float m = m_run[e >> 1];
-                pv[e] = (m == -INFINITY) ? 0.0f : exp2f(sc[nt][e] - m);
-                l_run[e >> 1] += pv[e];
-            }
-            const int kk = nt >> 1, hi2 = nt & 1;
-            pa[kk][0 + 2 * hi2] = ptx::pack_bf16(pv[0], pv[1]);
-            pa[kk][1 + 2 * hi2] = ptx::pack_bf16(pv[2], pv[3]);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-            for (int t = 0; t < A::ntile_o; t += 2) {
-                uint32_t vr[4];
-                const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                const int dim0 = part * A::dw + (t + (lane >> 4)) * 8;
-                ptx::ldmatrix_x4_trans(vr, vb + key * A::krow + head_off + dim0 * 2);
-                ptx::mma_bf16(oacc[t], pa[kk], vr[0], vr[1]);
-                ptx::mma_bf16(oacc[t + 1], pa[kk], vr[2], vr[3]);
-            }
-        }
-        if (st + 1 < nst) store_stage(st + 1);
-        __syncthreads();
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
-        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
-    }
+    constexpr int kb_row = HKV * kD;
+    AttAcc<HKV> acc;
+    attn_core<HKV>(qs, stage, mypos, mine, P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p,
+                   P.k_new + (int64_t)b * kb_row, P.v_new + (int64_t)b * kb_row, P.scale_log2,
+                   P.status, acc);
     // partial (m, l, O) of this CTA for the query heads of group g_w
     float* prow = P.part + ((int64_t)b * P.S2 + j) * P.H_q * (kD + 2);
 #pragma unroll
@@ -617,14 +472,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
         if (row < P.group) {
             float* rec = prow + (int64_t)(g_w * P.group + row) * (kD + 2);
             if (part == 0 && tq == 0) {
-                rec[0] = m_run[h];
-                rec[1] = l_run[h];
+                rec[0] = acc.m[h];
+                rec[1] = acc.l[h];
             }
 #pragma unroll
             for (int t = 0; t < A::ntile_o; ++t) {
                 const int dim = part * A::dw + t * 8 + 2 * tq;
-                rec[2 + dim] = oacc[t][2 * h];
-                rec[2 + dim + 1] = oacc[t][2 * h + 1];
+                rec[2 + dim] = acc.o[t][2 * h];
+                rec[2 + dim + 1] = acc.o[t][2 * h + 1];
             }
         }
     }

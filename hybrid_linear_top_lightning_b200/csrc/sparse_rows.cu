@@ -1,0 +1,113 @@
+// Sparse softmax attention over given index lists (lisa_sparse_attn) for many
+// query rows, bf16, head dim 128: one CTA per query row runs the gather and
+// tensor-core online softmax of attend_core.cuh over the row's count[b,t]
+// positions and writes the normalised output (LISA, arXiv 2607.19358v1,
+// Sec. 3.2 Eq. 1, the SA_M branch).  Positions outside [0, p] are masked out
+// and reported as LISA_ERR_DEVICE_BOUNDS through the status word.
+#include "attend_core.cuh"
+#include "lisa_fast.cuh"
+#include "lisa_internal.cuh"
+
+namespace lisa {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int kMaxList = 8192;  // positions per row held in shared memory
+
+struct SpParams {
+    int B, T, n_past, N_max, H_q, group, M;
+    float scale_log2;
+    const bf16* q;
+    const bf16* k;
+    const bf16* v;
+    const int32_t* idx;
+    const int32_t* count;
+    bf16* o;
+    unsigned* status;
+};
+
+template <int HKV>
+struct SpSmem {
+    static constexpr int q = 0;
+    static constexpr int pos = q + AttGeo<HKV>::qbytes;
+    static constexpr int stage = pos + kMaxList * 4;
+    static constexpr int total = stage + 2 * AttGeo<HKV>::stage_bytes;
+};
+
+template <int HKV>
+__global__ void __launch_bounds__(kAttThreads, 1) k_sparse_rows(const SpParams P) {
+    using A = AttGeo<HKV>;
+    using L = SpSmem<HKV>;
+    extern __shared__ __align__(128) uint8_t sp_raw[];
+    uint8_t* qs = sp_raw + L::q;
+    int* pos = reinterpret_cast<int*>(sp_raw + L::pos);
+    uint8_t* stage = sp_raw + L::stage;
+    const int row = blockIdx.x;
+    const int b = row / P.T, t = row % P.T;
+    const int p = P.n_past + t;
+    const int cnt = max(0, min(P.count[row], P.M));
+    for (int i = threadIdx.x; i < cnt; i += kAttThreads) pos[i] = P.idx[(int64_t)row * P.M + i];
+    attn_load_query<HKV>(qs, P.q + (int64_t)row * P.H_q * 128, P.group);
+    AttAcc<HKV> acc;
+    attn_core<HKV>(qs, stage, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1, nullptr, nullptr,
+                   P.scale_log2, P.status, acc);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gid = lane >> 2, tq = lane & 3;
+    const int g_w = warp / A::wph, part = warp % A::wph;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int r = gid + 8 * h;
+        if (r >= P.group) continue;
+        const float inv = acc.l[h] > 0.0f ? 1.0f / acc.l[h] : 0.0f;
+        bf16* orow = P.o + ((int64_t)row * P.H_q + g_w * P.group + r) * 128;
+#pragma unroll
+        for (int tt = 0; tt < A::ntile_o; ++tt) {
+            const int dim = part * A::dw + tt * 8 + 2 * tq;
+            *reinterpret_cast<__nv_bfloat162*>(orow + dim) =
+                __floats2bfloat162_rn(acc.o[tt][2 * h] * inv, acc.o[tt][2 * h + 1] * inv);
+        }
+    }
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+}  // namespace
+
+size_t fast_attention_ws_bytes(const Shape&, bool) { return kStatusBytes; }
+
+bool fast_attention_supported(const Shape& s, const void* q, const void* k, const void* v,
+                              bool dense) {
+    if (dense) return false;
+    if (s.dtype != LISA_BF16 || s.d != 128) return false;
+    if (!(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4) || s.group > 16 || s.M > kMaxList) return false;
+    return aligned16(q) && aligned16(k) && aligned16(v);
+}
+
+cudaError_t fast_attention(const Shape& s, const void* q, const void* k, const void* v,
+                           const int32_t* idx, const int32_t* count, void* o, void* ws,
+                           cudaStream_t st) {
+    SpParams P;
+    P.B = s.B; P.T = s.T; P.n_past = s.n_past; P.N_max = s.N_max; P.H_q = s.H_q;
+    P.group = s.group; P.M = s.M; P.scale_log2 = s.sm_scale * 1.4426950408889634f;
+    P.q = (const bf16*)q; P.k = (const bf16*)k; P.v = (const bf16*)v;
+    P.idx = idx; P.count = count; P.o = (bf16*)o; P.status = (unsigned*)ws;
+    static bool attrs[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attrs[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_sparse_rows<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, SpSmem<1>::total);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k_sparse_rows<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, SpSmem<2>::total);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k_sparse_rows<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SpSmem<4>::total);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attrs[dev] = true;
+    }
+    const dim3 grid(s.B * s.T);
+    switch (s.H_kv) {
+        case 1: k_sparse_rows<1><<<grid, kAttThreads, SpSmem<1>::total, st>>>(P); break;
+        case 2: k_sparse_rows<2><<<grid, kAttThreads, SpSmem<2>::total, st>>>(P); break;
+        default: k_sparse_rows<4><<<grid, kAttThreads, SpSmem<4>::total, st>>>(P); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace lisa
