@@ -320,6 +320,103 @@ def run_gpu(args, wl, rank, world, device):
     return line
 
 
+# ----------------------------------------------------------------------------- prefill
+def prefill_work(wl) -> dict:
+    """Algorithmic work of one causal prefill of wl.n tokens per sequence: causal
+    indexer pairs, key visits of the sparse attention (sum over rows of
+    min(M, t+1)) and the chunk GEMMs of the linear branch (flops, all B)."""
+    n, M = wl.n, wl.M
+    pairs = n * (n + 1) // 2
+    visits = sum(min(M, t + 1) for t in range(n))
+    indexer = pairs * wl.H_I * wl.d_I * 2
+    sparse = visits * wl.H_q * wl.d * 2 * 2
+    C = wl.chunk
+    nc = (n + C - 1) // C
+    # per chunk and KV head: K^T V (d x d x C); per query head: Q S (C x d x d),
+    # Q K^T (C x C x d, causal half) and P V (C x C x d, causal half)
+    lin = nc * (wl.H_kv * 2 * wl.d * wl.d * C
+                + wl.H_q * (2 * C * wl.d * wl.d + 2 * 2 * (C * (C + 1) // 2) * wl.d))
+    gather = visits * wl.H_kv * wl.d * 2 * 2
+    return dict(pairs=pairs * wl.B, visits=visits * wl.B, indexer=indexer * wl.B,
+                sparse=sparse * wl.B, linear=lin * wl.B, gather_bytes=gather * wl.B,
+                total=(indexer + sparse + lin) * wl.B)
+
+
+def run_prefill(args, wl, device):
+    """Times one whole-module prefill (lisa_prefill) of the 7B-shaped layer and,
+    separately, each of its four stages; L2 is flushed before every timed call."""
+    import torch
+
+    from hybrid_linear_top_lightning_b200 import inputs, lisa
+
+    gen = inputs.Generator(wl)
+    n, B, bf = wl.n, wl.B, torch.bfloat16
+
+    def dv(name, dt=bf):
+        return torch.from_numpy(gen.batch(name, 0, n)).to(dt).to(device)
+
+    q, k, v, qI, kI = dv("q"), dv("k"), dv("v"), dv("q_I"), dv("k_I")
+    w, gl = dv("w", torch.float32), dv("gate")
+    D = lisa.make_dims(B, n, 0, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                       chunk=wl.chunk)
+    S = torch.zeros(B, wl.H_kv, wl.d, wl.d, device=device)
+    o = torch.empty(B, n, wl.H_q, wl.d, dtype=bf, device=device)
+    o_sp, o_lin = torch.empty_like(o), torch.empty_like(o)
+    idx = torch.empty(B, n, wl.M, dtype=torch.int32, device=device)
+    cnt = torch.empty(B, n, dtype=torch.int32, device=device)
+    ws = lisa.workspace(D, lisa.LISA_OP_PREFILL, device)
+    args_p = lisa.prefill_args(q, k, v, qI, kI, w, wl.H_I, q, k, v, gl, S, None, o, idx, cnt)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    stages = {
+        "whole": lambda: lisa.lisa_prefill(D, args_p, ws, stream),
+        "topm": lambda: lisa.lisa_topm(D, qI, kI, w, wl.H_I, idx, cnt, ws, stream),
+        "sparse_attn": lambda: lisa.lisa_sparse_attn(D, q, k, v, idx, cnt, o_sp, ws, stream),
+        "linear": lambda: lisa.lisa_linear_prefill(D, q, k, v, S, None, o_lin, ws, stream),
+        "gate": lambda: lisa.lisa_gate_fuse(D, gl, o_lin, o_sp, o, stream),
+    }
+    steps = max(1, args.prefill_steps)
+    times = {}
+    for name, fn in stages.items():
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1)  # evict the previous call's data from L2
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            fn()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a_.elapsed_time(b_))
+        times[name] = statistics.median(ts)
+        assert lisa.lisa_check_status(ws, stream) == lisa.LISA_OK
+    work = prefill_work(wl)
+    _, tc_burst, peak_kind = _peaks()
+    whole_s = times["whole"] / 1e3
+    idx_tf = work["indexer"] / (times["topm"] / 1e3) / 1e12
+    lin_tf = work["linear"] / (times["linear"] / 1e3) / 1e12
+    return {
+        "workload": wl.name, "B": B, "n": n, "M": wl.M, "H_q": wl.H_q, "H_kv": wl.H_kv,
+        "value": B * n / whole_s, "unit": "tok/s", "ms": times["whole"], "steps": steps,
+        "stage_ms": {k_: v_ for k_, v_ in times.items() if k_ != "whole"},
+        "gpu_launches_per_prefill": 7,
+        "l2": "256 MB buffer written before every timed call",
+        "work": {"indexer_gflop": work["indexer"] / 1e9, "sparse_gflop": work["sparse"] / 1e9,
+                 "linear_gflop": work["linear"] / 1e9, "gather_gb": work["gather_bytes"] / 1e9},
+        "roofline": {
+            "bound": "tensor", "unit": "TFLOP/s", "peak": tc_burst, "peak_kind": peak_kind,
+            "achieved": work["total"] / whole_s / 1e12,
+            "frac": work["total"] / whole_s / 1e12 / tc_burst,
+            "indexer_tflops_incl_select": idx_tf, "indexer_frac_incl_select": idx_tf / tc_burst,
+            "linear_tflops": lin_tf, "linear_frac": lin_tf / tc_burst,
+            "sparse_gather_gbs": work["gather_bytes"] / (times["sparse_attn"] / 1e3) / 1e9,
+            "traffic": None},
+    }
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_decode_sample(wl, seqs: int, budget_s: float):
     """Time the oracle's decode step on `seqs` sequences of the workload, repeated
@@ -377,6 +474,8 @@ def main():
     ap.add_argument("--rotate", type=int, default=4,
                     help="copies of the decode state used in rotation (inputs larger than L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=3,
+                    help="timed calls per stage of the 7B prefill line (0: skip it)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -404,6 +503,8 @@ def main():
                                 device_id=device)
     try:
         line = run_gpu(args, wl, rank, world, device)
+        if args.prefill_steps > 0:
+            line["prefill"] = run_prefill(args, inputs.PREFILL_7B, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             tok_s, cores, note = oracle_decode_sample(wl, seqs=2, budget_s=args.cpu_seconds)
             line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores,

@@ -69,6 +69,28 @@ DecodeWs decode_ws(const Shape& s) {
     return w;
 }
 
+size_t workspace_bytes(const Shape& s, int op);
+
+// Whole-module prefill: the sub-operations run one after another on the
+// stream and share [status | scratch]; the intermediates follow the scratch.
+struct PrefillWs { size_t scratch_end, idx, count, o_sp, o_lin, end; };
+PrefillWs prefill_ws(const Shape& s) {
+    PrefillWs w;
+    size_t scratch = workspace_bytes(s, LISA_OP_TOPM);
+    const size_t lin = workspace_bytes(s, LISA_OP_LINEAR_PREFILL);
+    const size_t att = workspace_bytes(s, LISA_OP_SPARSE_ATTN);
+    if (lin > scratch) scratch = lin;
+    if (att > scratch) scratch = att;
+    const size_t esz = s.dtype == LISA_BF16 ? 2 : 4;
+    w.scratch_end = align256(scratch);
+    w.idx = w.scratch_end;
+    w.count = w.idx + align256(sizeof(int32_t) * (size_t)s.B * s.T * s.M);
+    w.o_sp = w.count + align256(sizeof(int32_t) * (size_t)s.B * s.T);
+    w.o_lin = w.o_sp + align256(esz * (size_t)s.B * s.T * s.H_q * s.d);
+    w.end = w.o_lin + align256(esz * (size_t)s.B * s.T * s.H_q * s.d);
+    return w;
+}
+
 lisa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
     if (!ws) return LISA_ERR_WORKSPACE;
     if (((uintptr_t)ws & 255) != 0) return LISA_ERR_WORKSPACE;
@@ -97,6 +119,7 @@ size_t workspace_bytes(const Shape& s, int op) {
             size_t fast = fast_decode_ws_bytes(s);
             return need > fast ? need : fast;
         }
+        case LISA_OP_PREFILL: return prefill_ws(s).end;
         default: return 0;
     }
 }
@@ -123,7 +146,7 @@ extern "C" {
 lisa_status lisa_workspace_size(const lisa_dims* dims, int op, size_t* bytes) {
     LISA_TRY(check_dims(dims));
     if (!bytes) return LISA_ERR_INVALID_ARG;
-    if (op < LISA_OP_TOPM || op > LISA_OP_DENSE_ATTN) return LISA_ERR_INVALID_ARG;
+    if (op < LISA_OP_TOPM || op > LISA_OP_PREFILL) return LISA_ERR_INVALID_ARG;
     *bytes = workspace_bytes(resolve(*dims), op);
     return LISA_OK;
 }
@@ -257,6 +280,35 @@ lisa_status lisa_decode_step(const lisa_dims* dims, const lisa_decode_args* a, v
     LISA_CUDA(generic_attention(s, a->q, a->k_cache, a->v_cache, idx, count, o_sp, true,
                                 (unsigned*)ws, st));
     return cuda_status(generic_gate(s, a->gate_logit_lin, o_lin, true, o_sp, true, a->o, st));
+}
+
+lisa_status lisa_prefill(const lisa_dims* dims, const lisa_prefill_args* a, void* ws,
+                         size_t ws_bytes, void* stream) {
+    LISA_TRY(check_dims(dims));
+    if (!a) return LISA_ERR_INVALID_ARG;
+    LISA_TRY(check_w_stride(*dims, a->w_tok_stride));
+    const Shape s = resolve(*dims);
+    if ((int64_t)s.B * s.T == 0) return LISA_OK;
+    if (!a->q || !a->k_cache || !a->v_cache || !a->q_I || !a->k_I_cache || !a->w || !a->q_L ||
+        !a->k_L || !a->v_L || !a->gate_logit_lin || !a->S || !a->o)
+        return LISA_ERR_INVALID_ARG;
+    if (s.phi == LISA_PHI_ELU1_NORM && !a->z) return LISA_ERR_INVALID_ARG;
+    if (s.chunk <= 0) return LISA_ERR_INVALID_ARG;
+    const PrefillWs lay = prefill_ws(s);
+    LISA_TRY(check_ws(ws, ws_bytes, lay.end));
+    char* base = (char*)ws;
+    int32_t* idx = a->idx ? a->idx : (int32_t*)(base + lay.idx);
+    int32_t* count = a->count ? a->count : (int32_t*)(base + lay.count);
+    void* o_sp = base + lay.o_sp;
+    void* o_lin = base + lay.o_lin;
+    // the sub-operations see [status | scratch] as their own workspace
+    LISA_TRY(lisa_topm(dims, a->q_I, a->k_I_cache, a->w, a->w_tok_stride, idx, count, ws,
+                       lay.scratch_end, stream));
+    LISA_TRY(lisa_sparse_attn(dims, a->q, a->k_cache, a->v_cache, idx, count, o_sp, ws,
+                              lay.scratch_end, stream));
+    LISA_TRY(lisa_linear_prefill(dims, a->q_L, a->k_L, a->v_L, a->S, a->z, o_lin, ws,
+                                 lay.scratch_end, stream));
+    return lisa_gate_fuse(dims, a->gate_logit_lin, o_lin, o_sp, a->o, stream);
 }
 
 lisa_status lisa_check_status(void* ws, void* stream) {

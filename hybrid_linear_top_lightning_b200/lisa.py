@@ -34,13 +34,14 @@ LISA_OP_SPARSE_ATTN = 1
 LISA_OP_LINEAR_PREFILL = 2
 LISA_OP_DECODE_STEP = 3
 LISA_OP_DENSE_ATTN = 4
+LISA_OP_PREFILL = 5
 
 # Every symbol the header declares.
 EXPORTS = (
     "lisa_index_scores", "lisa_topm", "lisa_sparse_attn", "lisa_linear_prefill",
     "lisa_linear_decode", "lisa_gate_fuse", "lisa_decode_step", "lisa_dense_attn",
     "lisa_workspace_size", "lisa_check_status", "lisa_status_string", "lisa_version",
-    "lisa_topm_noalloc",
+    "lisa_topm_noalloc", "lisa_prefill",
 )
 
 
@@ -54,6 +55,17 @@ class lisa_dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "T", "n_past", "N_max", "H_q", "H_kv", "d", "H_I", "H_Ik", "d_I", "M",
                  "chunk", "act_dtype", "phi")] + [("sm_scale", ctypes.c_float)]
+
+
+class lisa_prefill_args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("q_I", ctypes.c_void_p), ("k_I_cache", ctypes.c_void_p), ("w", ctypes.c_void_p),
+        ("w_tok_stride", ctypes.c_int64), ("q_L", ctypes.c_void_p), ("k_L", ctypes.c_void_p),
+        ("v_L", ctypes.c_void_p), ("gate_logit_lin", ctypes.c_void_p), ("S", ctypes.c_void_p),
+        ("z", ctypes.c_void_p), ("o", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+        ("count", ctypes.c_void_p),
+    ]
 
 
 class lisa_decode_args(ctypes.Structure):
@@ -94,6 +106,7 @@ def load() -> ctypes.CDLL:
         "lisa_workspace_size": [dp, ctypes.c_int, ctypes.POINTER(sz)],
         "lisa_check_status": [vp, vp],
         "lisa_topm_noalloc": [dp, vp, vp, vp, i64, vp, vp, vp],
+        "lisa_prefill": [dp, ctypes.POINTER(lisa_prefill_args), vp, sz, vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -221,6 +234,23 @@ def decode_args(q, k_new, v_new, q_I, k_I_new, w, w_tok_stride, q_L, k_L, v_L, g
     args._keep = (q, k_new, v_new, q_I, k_I_new, w, q_L, k_L, v_L, gate_logit_lin, k_cache,
                   v_cache, k_I_cache, S, z, o, idx, count)
     return args
+
+
+def prefill_args(q, k_cache, v_cache, q_I, k_I_cache, w, w_tok_stride, q_L, k_L, v_L,
+                 gate_logit_lin, S, z, o, idx=None, count=None) -> lisa_prefill_args:
+    args = lisa_prefill_args(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(q_I), _ptr(k_I_cache),
+                             _ptr(w), int(w_tok_stride), _ptr(q_L), _ptr(k_L), _ptr(v_L),
+                             _ptr(gate_logit_lin), _ptr(S), _ptr(z), _ptr(o), _ptr(idx),
+                             _ptr(count))
+    # the struct holds raw device pointers: keep the tensors alive with it
+    args._keep = (q, k_cache, v_cache, q_I, k_I_cache, w, q_L, k_L, v_L, gate_logit_lin, S, z,
+                  o, idx, count)
+    return args
+
+
+def lisa_prefill(dims, args: lisa_prefill_args, ws, stream=None):
+    _check(load().lisa_prefill(ctypes.byref(dims), ctypes.byref(args), _ptr(ws), ws.numel(),
+                               _stream(stream)), "lisa_prefill")
 
 
 def lisa_decode_step(dims, args: lisa_decode_args, ws, stream=None):

@@ -109,7 +109,8 @@ typedef enum lisa_op {
     LISA_OP_SPARSE_ATTN = 1,
     LISA_OP_LINEAR_PREFILL = 2,
     LISA_OP_DECODE_STEP = 3,
-    LISA_OP_DENSE_ATTN = 4
+    LISA_OP_DENSE_ATTN = 4,
+    LISA_OP_PREFILL = 5
 } lisa_op;
 
 /* Lightning Indexer scores (Sec. 3.2; the per-head score vector defined under
@@ -186,6 +187,35 @@ typedef struct lisa_decode_args {
  * attend over them; gate the two branches into o.  T must be 1. */
 LISA_API lisa_status lisa_decode_step(const lisa_dims* dims, const lisa_decode_args* args, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* Arguments of a whole-module prefill over the T tokens of a call.  All device
+ * pointers.  The caches must already hold positions [0, n_past + T). */
+typedef struct lisa_prefill_args {
+    const void* q;               /* [B,T,H_q,d]                                       */
+    const void* k_cache;         /* [B,N_max,H_kv,d]                                  */
+    const void* v_cache;         /* [B,N_max,H_kv,d]                                  */
+    const void* q_I;             /* [B,T,H_I,d_I]                                     */
+    const void* k_I_cache;       /* [B,N_max,H_Ik,d_I]                                */
+    const float* w;              /* indexer weights, see w_tok_stride                  */
+    int64_t w_tok_stride;        /* 0 or H_I                                          */
+    const void* q_L;             /* [B,T,H_q,d]                                       */
+    const void* k_L;             /* [B,T,H_kv,d]                                      */
+    const void* v_L;             /* [B,T,H_kv,d]                                      */
+    const void* gate_logit_lin;  /* [B,T,H_q]                                         */
+    float* S;                    /* [B,H_kv,d,d]  in: state before token 0, out: after  */
+    float* z;                    /* [B,H_kv,d]    in/out, NULL unless ELU1_NORM         */
+    void* o;                     /* [B,T,H_q,d]   output                               */
+    int32_t* idx;                /* [B,T,M] optional output (NULL: kept in workspace)  */
+    int32_t* count;              /* [B,T]   optional output                            */
+} lisa_prefill_args;
+
+/* The whole module over the T tokens of a call (Sec. 3.2 Eq. 1): indexer scores
+ * and top-M of every token, sparse attention over the selected rows, the
+ * linear branch in chunked form (advancing S and z), and the gate.  Equivalent
+ * to lisa_topm, lisa_sparse_attn, lisa_linear_prefill and lisa_gate_fuse in a
+ * row; intermediates live in the workspace (LISA_OP_PREFILL). */
+LISA_API lisa_status lisa_prefill(const lisa_dims* dims, const lisa_prefill_args* args, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Dense causal softmax attention over every cached position s <= p (Sec. 3.1,
  * the standard attention LISA replaces); the O(n) reference line. */

@@ -162,6 +162,54 @@ def _module_case(wl, T, rows):
         assert err <= TOL["bf16"], (name, err)
 
 
+def _whole_prefill_case(wl, T, rows, elu=False):
+    """The single whole-module entry point (lisa_prefill) vs the oracle module."""
+    gen = inputs.Generator(wl)
+    x = {n: gen.batch(n, 0, T) for n in ("q", "k", "v", "q_I", "k_I", "w", "gate")}
+    phi = lisa.LISA_PHI_ELU1_NORM if elu else lisa.LISA_PHI_IDENTITY
+    D = lisa.make_dims(wl.B, T, 0, T, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                       chunk=wl.chunk, phi=phi)
+    q, k, v = _dv(x["q"]), _dv(x["k"]), _dv(x["v"])
+    idx = torch.empty(wl.B, T, wl.M, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(wl.B, T, dtype=torch.int32, device="cuda")
+    S = torch.zeros(wl.B, wl.H_kv, wl.d, wl.d, device="cuda")
+    z = torch.zeros(wl.B, wl.H_kv, wl.d, device="cuda") if elu else None
+    o = torch.empty(wl.B, T, wl.H_q, wl.d, dtype=BF, device="cuda")
+    ws = lisa.workspace(D, lisa.LISA_OP_PREFILL)
+    args = lisa.prefill_args(q, k, v, _dv(x["q_I"]), _dv(x["k_I"]), _dv(x["w"], torch.float32),
+                             wl.H_I, q, k, v, _dv(x["gate"]), S, z, o, idx, cnt)
+    lisa.lisa_prefill(D, args, ws)
+    assert lisa.lisa_check_status(ws) == lisa.LISA_OK
+    Dr = ref.Dims(B=wl.B, T=T, n_past=0, N_max=T, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d, H_I=wl.H_I,
+                  H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M, phi=phi)
+    sc = ref.index_scores(Dr, x["q_I"], x["k_I"], x["w"], wl.H_I, rows=rows)
+    r_idx, r_cnt = ref.topm(Dr, sc, rows=rows)
+    g_idx, g_cnt = idx.cpu().numpy()[:, rows], cnt.cpu().numpy()[:, rows]
+    for b in range(wl.B):
+        check_topm(g_idx[b], g_cnt[b], r_idx[b], r_cnt[b], sc[b])
+    r_sp = ref.sparse_attn(Dr, x["q"], x["k"], x["v"], g_idx, g_cnt, rows=rows)
+    r_lin, r_S, r_z = ref.linear(Dr, x["q"], x["k"], x["v"], rows=rows)
+    r_o = ref.gate(Dr, x["gate"], r_lin, r_sp, rows=rows)
+    err = max_abs(o.float().cpu().numpy()[:, rows], r_o)
+    assert err <= TOL["bf16"], err
+    s_err = max_abs(S.cpu().numpy(), r_S)
+    assert s_err <= 1e-3 * max(1.0, float(np.abs(r_S).max())), s_err
+    if elu:
+        z_err = max_abs(z.cpu().numpy(), r_z)
+        assert z_err <= 1e-3 * max(1.0, float(np.abs(r_z).max())), z_err
+
+
+def test_prefill_entry_point_1p5b_every_row():
+    wl = inputs.PREFILL_1P5B
+    _whole_prefill_case(wl, wl.n, rows=np.arange(wl.n, dtype=np.int32))
+
+
+def test_prefill_entry_point_ragged_batched_elu():
+    wl = inputs.PREFILL_1P5B.with_(B=3, n=777)
+    _whole_prefill_case(wl, wl.n, rows=np.array([0, 1, 63, 64, 511, 512, 700, 776], np.int32),
+                        elu=True)
+
+
 def test_prefill_module_1p5b_every_row():
     wl = inputs.PREFILL_1P5B
     _module_case(wl, wl.n, rows=np.arange(wl.n, dtype=np.int32))
