@@ -476,6 +476,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=3,
                     help="timed calls per stage of the 7B prefill line (0: skip it)")
+    ap.add_argument("--prefill-n", type=int, default=0,
+                    help="prefill length of the prefill line (default: the 7B workload's 16384)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill line and print it (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -502,9 +506,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     try:
+        wl_p = inputs.PREFILL_7B
+        if args.prefill_n > 0:
+            wl_p = wl_p.with_(n=args.prefill_n, name=f"prefill_7b_n{args.prefill_n}")
+        if args.prefill_only:
+            if rank == 0:
+                print(json.dumps({"prefill": run_prefill(args, wl_p, device)}), flush=True)
+            return
         line = run_gpu(args, wl, rank, world, device)
         if args.prefill_steps > 0:
-            line["prefill"] = run_prefill(args, inputs.PREFILL_7B, device)
+            line["prefill"] = run_prefill(args, wl_p, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             tok_s, cores, note = oracle_decode_sample(wl, seqs=2, budget_s=args.cpu_seconds)
             line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores,

@@ -3,12 +3,18 @@
 // SA_M over the selected rows; GQA: query head h reads KV head h / group).
 //
 // The K and V rows of the positions (all KV heads of a position are one
-// contiguous row) are gathered in stages of 32 with 128-bit loads into
-// registers, one stage ahead of the math, and stored into padded shared-memory
-// rows.  Warp w serves KV head w / (8 / HKV) and a slice of the value dims;
-// the query heads of the group sit on the M side of mma m16n8k16 (rows past
-// the group are zero), keys on N for Q.K^T, keys on K for P.V; the softmax is
-// online (running max and sum per query head, base 2).
+// contiguous row) are gathered in stages by 16-byte asynchronous copies
+// (cp.async, through L2 only) into padded shared-memory rows, in a ring of
+// kAttStages stages of which all but the one being computed are in flight.
+//
+// Tensor-core mapping (mma m16n8k16, bf16 in, fp32 accumulate): the keys sit
+// on the M side and the (up to 8) query heads of a GQA group on N, so no MMA
+// row is padding.  Scores: S^T[key][head] = K[key,:] . Q[head,:], with the
+// query fragments held in registers for the whole row.  Output: the
+// probabilities are transposed in registers (movmatrix) and O^T[dim][head] +=
+// V^T[dim][key] P^T[key][head].  The warps serving one KV head split each
+// stage's keys 16 apiece and keep their own online-softmax state (base 2);
+// attn_core merges them at the end.
 #pragma once
 
 #include "lisa_internal.cuh"
@@ -18,201 +24,243 @@ namespace lisa {
 
 constexpr int kAttThreads = 256;
 constexpr int kAttWarps = kAttThreads / 32;
-constexpr int kGKeys = 32;             // keys per gather stage
-constexpr int kQRow = 128 * 2 + 16;    // padded shared-memory row of one query head (bytes)
+constexpr int kAttStages = 3;  // gather stages in the shared-memory ring
 
 template <int HKV>
 struct AttGeo {
     static constexpr int d = 128;
-    static constexpr int rowbytes = HKV * d * 2;      // one cached K (or V) row
-    static constexpr int krow = rowbytes + 16;        // padded shared-memory row
-    static constexpr int rpc = rowbytes / 16;         // 16-byte chunks per row
-    static constexpr int stage_bytes = kGKeys * 2 * krow;
-    static constexpr int chunks_per_thread = kGKeys * 2 * rpc / kAttThreads;
-    static constexpr int wph = kAttWarps / HKV;       // warps per KV head
-    static constexpr int dw = d / wph;                // output dims per warp
-    static constexpr int ntile_o = dw / 8;
-    static constexpr int qbytes = ((HKV * 16 * kQRow + 127) / 128) * 128;
+    static constexpr int rowbytes = HKV * d * 2;          // one cached K (or V) row
+    static constexpr int krow = rowbytes + 16;            // padded shared-memory row
+    static constexpr int rpc = rowbytes / 16;             // 16-byte chunks per row
+    static constexpr int wph = kAttWarps / HKV;           // warps per KV head
+    static constexpr int keys = 16 * wph;                 // keys per stage
+    static constexpr int tpk = kAttThreads / keys;        // copying threads per key
+    static constexpr int cpt = 2 * rpc / tpk;             // chunks per copying thread
+    static constexpr int stage_bytes = keys * 2 * krow;   // K rows, then V rows
+    static constexpr int ring_bytes = kAttStages * stage_bytes;
+    // merge scratch (in the ring after the loop): per warp O^T [8][128] + m[8] + l[8]
+    static constexpr int part_floats = 8 * d + 16;
+    static constexpr int res_off = kAttWarps * part_floats * 4;
+    // merged result: o [HKV*8][128], m [HKV*8], l [HKV*8] (floats)
+    static constexpr int res_bytes = (HKV * 8 * d + 2 * HKV * 8) * 4;
+    static_assert(cpt * tpk == 2 * rpc, "chunk split");
+    static_assert(res_off + res_bytes <= ring_bytes, "merge scratch fits in the ring");
 };
 
-// Per-warp result: running max (base 2) and sum of query rows gid and gid + 8,
-// and the un-normalised output tile of this warp's dims.
-template <int HKV>
-struct AttAcc {
-    float m[2];
-    float l[2];
-    float o[AttGeo<HKV>::ntile_o][4];
+// Merged result of attn_core, in shared memory (inside the ring): for KV head
+// g and head slot r of its group (r < 8), the base-2 running max m, the sum l
+// and the un-normalised output o[0..128) relative to m.
+struct AttResult {
+    const float* o;  // [(g * 8 + r) * 128 + dim]
+    const float* m;  // [g * 8 + r]
+    const float* l;  // [g * 8 + r]
 };
 
-// Loads the query heads of one row, [H_q][128] bf16 at q_row, into shared
-// memory: group g at rows g*16 .. g*16+group-1, the rest zero.
+// q_row: [H_q][128] bf16 (global) of this query row, `group` <= 8 heads per
+// KV head.  pos[0..cnt): positions (shared or global memory).  Position
+// `p_special` (if >= 0) is read from k_special / v_special instead of the
+// caches.  Positions outside [0, p_max] are masked out and reported through
+// `status`.  `ring` holds AttGeo<HKV>::ring_bytes bytes, `spos` (shared
+// memory) kAttStages * AttGeo<HKV>::keys ints.  Ends with a block barrier;
+// the result stays valid until the ring is reused.
 template <int HKV>
-__device__ __forceinline__ void attn_load_query(uint8_t* qs, const __nv_bfloat16* q_row, int group) {
-    for (int e = threadIdx.x; e < HKV * 16 * 16; e += kAttThreads) {
-        const int g = e / (16 * 16), r = (e / 16) % 16, c = e % 16;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < group) v = reinterpret_cast<const uint4*>(q_row + (int64_t)(g * group + r) * 128)[c];
-        *reinterpret_cast<uint4*>(qs + (g * 16 + r) * kQRow + c * 16) = v;
-    }
-}
-
-// pos[0..cnt): positions (shared memory).  Position `p_special` (if >= 0) is
-// read from k_special / v_special instead of the caches.  Positions outside
-// [0, p_max] are masked out and reported through `status`.
-template <int HKV>
-__device__ __forceinline__ void attn_core(const uint8_t* qs, uint8_t* stage, const int* pos, int cnt,
-                                          const __nv_bfloat16* k_cache, const __nv_bfloat16* v_cache,
-                                          int64_t row0,  // b * N_max
-                                          int p_max, int p_special, const __nv_bfloat16* k_special,
-                                          const __nv_bfloat16* v_special, float scale_log2,
-                                          unsigned* status, AttAcc<HKV>& acc) {
+__device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int group, uint8_t* ring,
+                                               int* spos, const int* pos, int cnt,
+                                               const __nv_bfloat16* k_cache,
+                                               const __nv_bfloat16* v_cache,
+                                               int64_t row0,  // b * N_max
+                                               int p_max, int p_special,
+                                               const __nv_bfloat16* k_special,
+                                               const __nv_bfloat16* v_special, float scale_log2,
+                                               unsigned* status) {
     using A = AttGeo<HKV>;
     using bf16 = __nv_bfloat16;
+    constexpr int GK = A::keys;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tq = lane & 3;
+    const int gid = lane >> 2, tq = lane & 3;
     const int g_w = warp / A::wph, part = warp % A::wph;
-    const int nst = (cnt + kGKeys - 1) / kGKeys;
+    const int key0 = part * 16;  // this warp's keys within a stage
+    const int nst = (cnt + GK - 1) / GK;
     constexpr int kb_row = HKV * 128;
 
-    uint4 rb[A::chunks_per_thread];
-    auto load_stage = [&](int st) {
+    // query fragments (B operand of the score MMA): head gid of group g_w,
+    // dims ks*16 + 2tq (+1) and + 8 (+9); heads past the group are zero
+    uint32_t qf[8][2];
+    {
+        const bool live = gid < group;
+        const uint32_t* qh =
+            reinterpret_cast<const uint32_t*>(q_row + (int64_t)(g_w * group + (live ? gid : 0)) * 128);
 #pragma unroll
-        for (int u = 0; u < A::chunks_per_thread; ++u) {
-            const int c = tid + u * kAttThreads;
-            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
-            const int which = w2 / A::rpc, off = w2 % A::rpc;
-            int jj = st * kGKeys + kk;
-            if (jj >= cnt) jj = st * kGKeys;  // pad with a listed row; masked below
-            int ps = pos[jj];
-            if (ps < 0 || ps > p_max) ps = 0;  // never dereference an out-of-range position
-            const bf16* src = (ps == p_special)
-                                  ? (which ? v_special : k_special)
-                                  : (which ? v_cache : k_cache) + (row0 + ps) * kb_row;
-            rb[u] = __ldg(reinterpret_cast<const uint4*>(src) + off);
+        for (int ks = 0; ks < 8; ++ks) {
+            qf[ks][0] = live ? __ldg(qh + ks * 8 + tq) : 0u;
+            qf[ks][1] = live ? __ldg(qh + ks * 8 + 4 + tq) : 0u;
         }
-    };
-    auto store_stage = [&](int st) {
-        uint8_t* dst = stage + (st & 1) * A::stage_bytes;
-#pragma unroll
-        for (int u = 0; u < A::chunks_per_thread; ++u) {
-            const int c = tid + u * kAttThreads;
-            const int kk = c / (2 * A::rpc), w2 = c % (2 * A::rpc);
-            const int which = w2 / A::rpc, off = w2 % A::rpc;
-            *reinterpret_cast<uint4*>(dst + which * kGKeys * A::krow + kk * A::krow + off * 16) = rb[u];
-        }
-    };
-
-    acc.m[0] = acc.m[1] = -INFINITY;
-    acc.l[0] = acc.l[1] = 0.0f;
-#pragma unroll
-    for (int t = 0; t < A::ntile_o; ++t)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc.o[t][e] = 0.0f;
-    const uint32_t q_base = ptx::smem_u32(qs + g_w * 16 * kQRow);
-    const uint32_t head_off = (uint32_t)(g_w * 128 * 2);
-
-    __syncthreads();  // the stage area is free and the query rows are in place
-    if (nst > 0) {
-        load_stage(0);
-        store_stage(0);
     }
-    __syncthreads();
+
+    // copy role: thread copies chunks sub, sub + tpk, ... of key ck's K and V rows
+    const int ck = tid / A::tpk, sub = tid % A::tpk;
+    auto issue_stage = [&](int st) {
+        uint8_t* dst = ring + (st % kAttStages) * A::stage_bytes;
+        int jj = st * GK + ck;
+        if (jj >= cnt) jj = st * GK;  // pad with a listed row; masked below
+        const int raw = pos[jj];
+        if (sub == 0) spos[(st % kAttStages) * GK + ck] = (st * GK + ck < cnt) ? raw : -1;
+        const int ps = (raw < 0 || raw > p_max) ? 0 : raw;  // never dereference out of range
+        const bf16* ksrc = (ps == p_special) ? k_special : k_cache + (row0 + ps) * kb_row;
+        const bf16* vsrc = (ps == p_special) ? v_special : v_cache + (row0 + ps) * kb_row;
+#pragma unroll
+        for (int u = 0; u < A::cpt; ++u) {
+            const int i = sub + u * A::tpk;
+            const int which = i / A::rpc, off = i % A::rpc;
+            const bf16* src = which ? vsrc : ksrc;
+            ptx::cp_async_16(dst + which * GK * A::krow + ck * A::krow + off * 16,
+                             reinterpret_cast<const uint4*>(src) + off);
+        }
+    };
+
+    float m[2] = {-INFINITY, -INFINITY};  // heads 2tq, 2tq + 1
+    float l[2] = {0.0f, 0.0f};
+    float o[8][4];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[t][e] = 0.0f;
+
+    const uint32_t head_off = (uint32_t)(g_w * 128 * 2);
+    // ldmatrix lane addressing: K as A (keys x dims), V as A^T (dims x keys)
+    const int ka_key = key0 + (lane & 7) + ((lane >> 3) & 1) * 8, ka_dim = (lane >> 4) * 8;
+    const int va_key = key0 + (lane & 7) + (lane >> 4) * 8, va_dim = ((lane >> 3) & 1) * 8;
+
+    __syncthreads();  // the ring is free
+#pragma unroll
+    for (int st = 0; st < kAttStages - 1; ++st) {
+        if (st < nst) issue_stage(st);
+        ptx::cp_async_commit();  // (possibly empty) group per stage keeps the count uniform
+    }
 #pragma unroll 1
     for (int st = 0; st < nst; ++st) {
-        if (st + 1 < nst) load_stage(st + 1);  // in flight while this stage computes
-        const uint32_t kb = ptx::smem_u32(stage + (st & 1) * A::stage_bytes);
-        const uint32_t vb = kb + kGKeys * A::krow;
-        float sc[4][4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[t][e] = 0.0f;
+        ptx::cp_async_wait_group<kAttStages - 2>();  // this thread's copies of stage st landed
+        // all copies of stage st are visible, and every warp is done with
+        // stage st - 1, whose slot the next issue reuses
+        __syncthreads();
+        if (st + kAttStages - 1 < nst) issue_stage(st + kAttStages - 1);
+        ptx::cp_async_commit();
+        const uint32_t kb = ptx::smem_u32(ring + (st % kAttStages) * A::stage_bytes);
+        const uint32_t vb = kb + GK * A::krow;
+        const int* stpos = spos + (st % kAttStages) * GK;
+
+        // scores of this warp's 16 keys x 8 heads (two accumulation chains)
+        float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int ks = 0; ks < 8; ks += 2) {
-            uint32_t qa0[4], qa1[4];
-            {
-                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int col = ks * 16 + (lane >> 4) * 8;
-                ptx::ldmatrix_x4(qa0, q_base + row * kQRow + col * 2);
-                ptx::ldmatrix_x4(qa1, q_base + row * kQRow + (col + 16) * 2);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                uint32_t kr[4];
-                const int key = nt * 8 + (lane & 7);
-                const int dim0 = ks * 16 + (lane >> 3) * 8;
-                ptx::ldmatrix_x4(kr, kb + key * A::krow + head_off + dim0 * 2);
-                ptx::mma_bf16(sc[nt], qa0, kr[0], kr[1]);
-                ptx::mma_bf16(sc[nt], qa1, kr[2], kr[3]);
-            }
+            uint32_t a0[4], a1[4];
+            ptx::ldmatrix_x4(a0, kb + ka_key * A::krow + head_off + (ks * 16 + ka_dim) * 2);
+            ptx::ldmatrix_x4(a1, kb + ka_key * A::krow + head_off + ((ks + 1) * 16 + ka_dim) * 2);
+            ptx::mma_bf16(s0, a0, qf[ks][0], qf[ks][1]);
+            ptx::mma_bf16(s1, a1, qf[ks + 1][0], qf[ks + 1][1]);
         }
-        float mt[2] = {-INFINITY, -INFINITY};
+        // element e: key key0 + gid + 8 (e >> 1), head 2tq + (e & 1)
+        float v[4];
         bool bad = false;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int r = 0; r < 2; ++r) {
+            const int ps = stpos[key0 + gid + 8 * r];  // -1 past the list
+            const bool listed = st * GK + key0 + gid + 8 * r < cnt;
+            const bool ok = listed && ps >= 0 && ps <= p_max;
+            bad |= listed && !ok;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = st * kGKeys + nt * 8 + 2 * tq + (e & 1);
-                float v = sc[nt][e] * scale_log2;
-                if (j >= cnt) {
-                    v = -INFINITY;
-                } else {
-                    const int ps = pos[j];
-                    if (ps < 0 || ps > p_max) { v = -INFINITY; bad = true; }
-                }
-                sc[nt][e] = v;
-                mt[e >> 1] = fmaxf(mt[e >> 1], v);
-            }
+            for (int h = 0; h < 2; ++h)
+                v[2 * r + h] = ok ? (s0[2 * r + h] + s1[2 * r + h]) * scale_log2 : -INFINITY;
+        }
         if (bad) record_error(status, kDevBounds);
         float corr[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 1));
-            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 2));
-            const float m_new = fmaxf(acc.m[h], mt[h]);
-            corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(acc.m[h] - m_new);
-            acc.m[h] = m_new;
-            acc.l[h] *= corr[h];
+            float mt = fmaxf(v[h], v[2 + h]);
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+            const float m_new = fmaxf(m[h], mt);
+            corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m[h] - m_new);
+            m[h] = m_new;
+            l[h] *= corr[h];
+        }
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float mm = m[e & 1];
+            p[e] = (mm == -INFINITY) ? 0.0f : exp2f(v[e] - mm);
+            l[e & 1] += p[e];
         }
 #pragma unroll
-        for (int t = 0; t < A::ntile_o; ++t) {
-            acc.o[t][0] *= corr[0]; acc.o[t][1] *= corr[0];
-            acc.o[t][2] *= corr[1]; acc.o[t][3] *= corr[1];
+        for (int t = 0; t < 8; ++t) {
+            o[t][0] *= corr[0]; o[t][1] *= corr[1];
+            o[t][2] *= corr[0]; o[t][3] *= corr[1];
         }
-        uint32_t pa[2][4];
+        // P^T fragments (keys x heads) -> B operand (k = keys, n = heads)
+        const uint32_t b0 = ptx::movmatrix_trans(ptx::pack_bf16(p[0], p[1]));
+        const uint32_t b1 = ptx::movmatrix_trans(ptx::pack_bf16(p[2], p[3]));
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            float pv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float m = acc.m[e >> 1];
-                pv[e] = (m == -INFINITY) ? 0.0f : exp2f(sc[nt][e] - m);
-                acc.l[e >> 1] += pv[e];
-            }
-            const int kk = nt >> 1, hi2 = nt & 1;
-            pa[kk][0 + 2 * hi2] = ptx::pack_bf16(pv[0], pv[1]);
-            pa[kk][1 + 2 * hi2] = ptx::pack_bf16(pv[2], pv[3]);
+        for (int t = 0; t < 8; ++t) {
+            uint32_t va[4];
+            ptx::ldmatrix_x4_trans(va, vb + va_key * A::krow + head_off + (t * 16 + va_dim) * 2);
+            ptx::mma_bf16(o[t], va, b0, b1);
         }
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-            for (int t = 0; t < A::ntile_o; t += 2) {
-                uint32_t vr[4];
-                const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                const int dim0 = part * A::dw + (t + (lane >> 4)) * 8;
-                ptx::ldmatrix_x4_trans(vr, vb + key * A::krow + head_off + dim0 * 2);
-                ptx::mma_bf16(acc.o[t], pa[kk], vr[0], vr[1]);
-                ptx::mma_bf16(acc.o[t + 1], pa[kk], vr[2], vr[3]);
-            }
-        }
-        if (st + 1 < nst) store_stage(st + 1);
-        __syncthreads();
     }
+    ptx::cp_async_wait_all();
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        acc.l[h] += __shfl_xor_sync(0xffffffffu, acc.l[h], 1);
-        acc.l[h] += __shfl_xor_sync(0xffffffffu, acc.l[h], 2);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 4);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
+        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
     }
+    __syncthreads();  // every warp is done with the ring
+
+    // ---- merge the warps of each KV head
+    float* ringf = reinterpret_cast<float*>(ring);
+    float* pw = ringf + warp * A::part_floats;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            pw[(2 * tq + (e & 1)) * 128 + t * 16 + gid + 8 * (e >> 1)] = o[t][e];
+    if (gid == 0) {
+        pw[8 * 128 + 2 * tq] = m[0];
+        pw[8 * 128 + 2 * tq + 1] = m[1];
+        pw[8 * 128 + 8 + 2 * tq] = l[0];
+        pw[8 * 128 + 8 + 2 * tq + 1] = l[1];
+    }
+    __syncthreads();
+    float* res = reinterpret_cast<float*>(ring + A::res_off);
+    float* res_m = res + HKV * 8 * 128;
+    float* res_l = res_m + HKV * 8;
+    for (int e = tid; e < HKV * 8 * 128; e += kAttThreads) {
+        const int hs = e / 128, dim = e % 128;  // hs = g * 8 + r
+        const int g = hs / 8, r = hs % 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < A::wph; ++k)
+            M = fmaxf(M, ringf[(g * A::wph + k) * A::part_floats + 8 * 128 + r]);
+        float L = 0.0f, O = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < A::wph; ++k) {
+                const float* q = ringf + (g * A::wph + k) * A::part_floats;
+                const float mk = q[8 * 128 + r];
+                if (mk == -INFINITY) continue;
+                const float w = exp2f(mk - M);
+                L = fmaf(q[8 * 128 + 8 + r], w, L);
+                O = fmaf(q[r * 128 + dim], w, O);
+            }
+        }
+        res[e] = O;
+        if (dim == 0) {
+            res_m[hs] = M;
+            res_l[hs] = L;
+        }
+    }
+    __syncthreads();
+    return AttResult{res, res_m, res_l};
 }
 
 }  // namespace lisa

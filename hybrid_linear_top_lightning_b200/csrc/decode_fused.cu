@@ -382,17 +382,21 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
 template <int HKV>
 struct Att : AttGeo<HKV> {
     using G = AttGeo<HKV>;
-    // shared memory: histogram, barrier, broadcasts, selected positions,
-    // queries, candidate lists, gather stages (the score row during selection)
-    static constexpr int hist = 0;                     // u32[4096]
-    static constexpr int bar = hist + 4096 * 4;
-    static constexpr int bc = bar + 16;                 // int[128]
+    // shared memory: the gather ring first, which during selection holds the
+    // histogram, the candidate lists and (when it fits) the score row; then
+    // the barrier, broadcasts, selected positions and stage positions
+    static constexpr int ring = 0;
+    static constexpr int hist = ring;                                  // u32[4096]
+    static constexpr int cand = hist + 4096 * 4;                       // uint2[8][kCandCap]
+    static constexpr int row = cand + kAttWarps * kCandCap * 8;        // float[key_cap]
+    static constexpr int key_cap = (G::ring_bytes - row) / 4 - 32;     // scores that fit
+    static constexpr int bar = ring + G::ring_bytes;
+    static constexpr int bc = bar + 16;                                // int[128]
     static constexpr int mypos = bc + 128 * 4;
-    static constexpr int q = mypos + kMaxPer * 4;
-    static constexpr int cand = q + G::qbytes;          // uint2[8][kCandCap]
-    static constexpr int stage = cand + kAttWarps * kCandCap * 8;
-    static constexpr int total = stage + 2 * G::stage_bytes;
-    static constexpr int key_cap = 2 * G::stage_bytes / 4 - 32;  // scores that fit in the stages
+    static constexpr int spos = mypos + kMaxPer * 4;                   // int[stages][keys]
+    static constexpr int total = spos + kAttStages * G::keys * 4;
+    static_assert(row < G::ring_bytes, "selection scratch must fit in the gather ring");
+    static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
 
 template <int HKV>
@@ -403,17 +407,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     uint64_t* rowbar = reinterpret_cast<uint64_t*>(att_raw + A::bar);
     int* bc = reinterpret_cast<int*>(att_raw + A::bc);
     int* mypos = reinterpret_cast<int*>(att_raw + A::mypos);
-    uint8_t* qs = att_raw + A::q;
-    uint8_t* stage = att_raw + A::stage;
+    uint8_t* stage = att_raw + A::ring;
+    float* row_smem = reinterpret_cast<float*>(att_raw + A::row);
+    int* spos = reinterpret_cast<int*>(att_raw + A::spos);
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gid = lane >> 2, tq = lane & 3;
+    const int tid = threadIdx.x;
     const int b = blockIdx.x / P.S2, j = blockIdx.x % P.S2;
     const int n = P.n, p = n - 1;
     ptx::pdl_launch_dependents();
 
     // ---- prologue (inputs only; nothing written by the scan kernel)
-    attn_load_query<HKV>(qs, P.q + (int64_t)b * P.H_q * kD, P.group);
     if (tid == 0) {
         ptx::mbar_init(rowbar, 1);
         ptx::fence_mbar_init();
@@ -439,13 +442,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
             const int bytes = ((n + 3) / 4) * 16;
             ptx::mbar_arrive_expect_tx(rowbar, bytes);
             for (int off = 0; off < bytes; off += 16384)
-                ptx::bulk_load(stage + off, srow + off / 4, min(16384, bytes - off), rowbar);
+                ptx::bulk_load(reinterpret_cast<uint8_t*>(row_smem) + off, srow + off / 4,
+                               min(16384, bytes - off), rowbar);
         }
         SelectSmem sel;
         sel.hist = hist;
         sel.bc = bc;
         sel.cand = reinterpret_cast<uint2*>(att_raw + A::cand);
-        row_topm(resident ? reinterpret_cast<const float*>(stage) : srow, resident, n, P.M,
+        row_topm(resident ? row_smem : srow, resident, n, P.M,
                  P.hist + (int64_t)b * 4096, sel, lo, hi, mypos, resident ? rowbar : nullptr,
                  P.status);
     }
@@ -458,32 +462,23 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     if (P.count && j == 0 && tid == 0) P.count[b] = cnt;
 
     // ---- gather + attention over this CTA's positions
-    const int g_w = warp / A::wph, part = warp % A::wph;
     constexpr int kb_row = HKV * kD;
-    AttAcc<HKV> acc;
-    attn_core<HKV>(qs, stage, mypos, mine, P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p,
-                   P.k_new + (int64_t)b * kb_row, P.v_new + (int64_t)b * kb_row, P.scale_log2,
-                   P.status, acc);
-    // partial (m, l, O) of this CTA for the query heads of group g_w
+    const AttResult r = attn_core<HKV>(P.q + (int64_t)b * P.H_q * kD, P.group, stage, spos, mypos,
+                                       mine, P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p,
+                                       P.k_new + (int64_t)b * kb_row,
+                                       P.v_new + (int64_t)b * kb_row, P.scale_log2, P.status);
+    // partial (m, l, O) of this CTA for every query head
     float* prow = P.part + ((int64_t)b * P.S2 + j) * P.H_q * (kD + 2);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int row = gid + 8 * h;
-        if (row < P.group) {
-            float* rec = prow + (int64_t)(g_w * P.group + row) * (kD + 2);
-            if (part == 0 && tq == 0) {
-                rec[0] = acc.m[h];
-                rec[1] = acc.l[h];
-            }
-#pragma unroll
-            for (int t = 0; t < A::ntile_o; ++t) {
-                const int dim = part * A::dw + t * 8 + 2 * tq;
-                rec[2 + dim] = acc.o[t][2 * h];
-                rec[2 + dim + 1] = acc.o[t][2 * h + 1];
-            }
+    for (int e = tid; e < P.H_q * kD; e += kAttThreads) {
+        const int h = e / kD, dim = e % kD;
+        const int hs = (h / P.group) * 8 + h % P.group;
+        float* rec = prow + (int64_t)h * (kD + 2);
+        rec[2 + dim] = r.o[hs * kD + dim];
+        if (dim == 0) {
+            rec[0] = r.m[hs];
+            rec[1] = r.l[hs];
         }
     }
-
 }
 
 // ============================================================================ K3: combine
@@ -592,7 +587,7 @@ size_t fast_decode_ws_bytes(const Shape& s) {
 
 bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
     if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD || s.d_I != kDI || s.H_Ik != 1) return false;
-    if (s.H_I > 8 || s.group > 16 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
+    if (s.H_I > 8 || s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
     if (s.L < 1 || s.M < 1 || s.B < 1) return false;
     const Plan pl = make_plan(s);
     if (pl.per > kMaxPer) return false;

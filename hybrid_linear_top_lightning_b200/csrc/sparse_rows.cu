@@ -12,8 +12,6 @@ namespace lisa {
 namespace {
 
 using bf16 = __nv_bfloat16;
-constexpr int kMaxList = 8192;  // positions per row held in shared memory
-
 struct SpParams {
     int B, T, n_past, N_max, H_q, group, M;
     float scale_log2;
@@ -28,44 +26,33 @@ struct SpParams {
 
 template <int HKV>
 struct SpSmem {
-    static constexpr int q = 0;
-    static constexpr int pos = q + AttGeo<HKV>::qbytes;
-    static constexpr int stage = pos + kMaxList * 4;
-    static constexpr int total = stage + 2 * AttGeo<HKV>::stage_bytes;
+    static constexpr int spos = 0;                                     // int[stages][keys]
+    static constexpr int ring = (kAttStages * AttGeo<HKV>::keys * 4 + 127) / 128 * 128;
+    static constexpr int total = ring + AttGeo<HKV>::ring_bytes;
+    static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
 
 template <int HKV>
 __global__ void __launch_bounds__(kAttThreads, 1) k_sparse_rows(const SpParams P) {
-    using A = AttGeo<HKV>;
     using L = SpSmem<HKV>;
     extern __shared__ __align__(128) uint8_t sp_raw[];
-    uint8_t* qs = sp_raw + L::q;
-    int* pos = reinterpret_cast<int*>(sp_raw + L::pos);
-    uint8_t* stage = sp_raw + L::stage;
+    int* spos = reinterpret_cast<int*>(sp_raw + L::spos);
     const int row = blockIdx.x;
     const int b = row / P.T, t = row % P.T;
     const int p = P.n_past + t;
     const int cnt = max(0, min(P.count[row], P.M));
-    for (int i = threadIdx.x; i < cnt; i += kAttThreads) pos[i] = P.idx[(int64_t)row * P.M + i];
-    attn_load_query<HKV>(qs, P.q + (int64_t)row * P.H_q * 128, P.group);
-    AttAcc<HKV> acc;
-    attn_core<HKV>(qs, stage, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1, nullptr, nullptr,
-                   P.scale_log2, P.status, acc);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gid = lane >> 2, tq = lane & 3;
-    const int g_w = warp / A::wph, part = warp % A::wph;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int r = gid + 8 * h;
-        if (r >= P.group) continue;
-        const float inv = acc.l[h] > 0.0f ? 1.0f / acc.l[h] : 0.0f;
-        bf16* orow = P.o + ((int64_t)row * P.H_q + g_w * P.group + r) * 128;
-#pragma unroll
-        for (int tt = 0; tt < A::ntile_o; ++tt) {
-            const int dim = part * A::dw + tt * 8 + 2 * tq;
-            *reinterpret_cast<__nv_bfloat162*>(orow + dim) =
-                __floats2bfloat162_rn(acc.o[tt][2 * h] * inv, acc.o[tt][2 * h + 1] * inv);
-        }
+    const int* pos = P.idx + (int64_t)row * P.M;  // read through L1 by the gather
+    const AttResult r = attn_core<HKV>(P.q + (int64_t)row * P.H_q * 128, P.group, sp_raw + L::ring,
+                                       spos, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1,
+                                       nullptr, nullptr, P.scale_log2, P.status);
+    // normalised output, two dims per thread
+    for (int e = threadIdx.x; e < P.H_q * 64; e += kAttThreads) {
+        const int h = e / 64, dim = (e % 64) * 2;
+        const int hs = (h / P.group) * 8 + h % P.group;
+        const float lsum = r.l[hs];
+        const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+        *reinterpret_cast<__nv_bfloat162*>(P.o + ((int64_t)row * P.H_q + h) * 128 + dim) =
+            __floats2bfloat162_rn(r.o[hs * 128 + dim] * inv, r.o[hs * 128 + dim + 1] * inv);
     }
 }
 
@@ -79,7 +66,7 @@ bool fast_attention_supported(const Shape& s, const void* q, const void* k, cons
                               bool dense) {
     if (dense) return false;
     if (s.dtype != LISA_BF16 || s.d != 128) return false;
-    if (!(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4) || s.group > 16 || s.M > kMaxList) return false;
+    if (!(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4) || s.group > 8) return false;
     return aligned16(q) && aligned16(k) && aligned16(v);
 }
 
