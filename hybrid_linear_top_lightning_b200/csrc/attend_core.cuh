@@ -99,11 +99,14 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
 
     // copy role: thread copies chunks sub, sub + tpk, ... of key ck's K and V rows
     const int ck = tid / A::tpk, sub = tid % A::tpk;
-    auto issue_stage = [&](int st) {
+    // position of key ck of stage st (a listed row pads the last stage; masked below)
+    auto load_pos = [&](int st) -> int {
+        if (st * GK >= cnt) return 0;
+        const int jj = st * GK + ck;
+        return pos[jj < cnt ? jj : st * GK];
+    };
+    auto issue_stage = [&](int st, int raw) {
         uint8_t* dst = ring + (st % kAttStages) * A::stage_bytes;
-        int jj = st * GK + ck;
-        if (jj >= cnt) jj = st * GK;  // pad with a listed row; masked below
-        const int raw = pos[jj];
         if (sub == 0) spos[(st % kAttStages) * GK + ck] = (st * GK + ck < cnt) ? raw : -1;
         const int ps = (raw < 0 || raw > p_max) ? 0 : raw;  // never dereference out of range
         const bf16* ksrc = (ps == p_special) ? k_special : k_cache + (row0 + ps) * kb_row;
@@ -134,17 +137,20 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
     __syncthreads();  // the ring is free
 #pragma unroll
     for (int st = 0; st < kAttStages - 1; ++st) {
-        if (st < nst) issue_stage(st);
+        if (st < nst) issue_stage(st, load_pos(st));
         ptx::cp_async_commit();  // (possibly empty) group per stage keeps the count uniform
     }
+    // the positions of the next stage to issue are loaded one iteration ahead
+    int next_pos = load_pos(kAttStages - 1);
 #pragma unroll 1
     for (int st = 0; st < nst; ++st) {
         ptx::cp_async_wait_group<kAttStages - 2>();  // this thread's copies of stage st landed
         // all copies of stage st are visible, and every warp is done with
         // stage st - 1, whose slot the next issue reuses
         __syncthreads();
-        if (st + kAttStages - 1 < nst) issue_stage(st + kAttStages - 1);
+        if (st + kAttStages - 1 < nst) issue_stage(st + kAttStages - 1, next_pos);
         ptx::cp_async_commit();
+        next_pos = load_pos(st + kAttStages);
         const uint32_t kb = ptx::smem_u32(ring + (st % kAttStages) * A::stage_bytes);
         const uint32_t vb = kb + GK * A::krow;
         const int* stpos = spos + (st % kAttStages) * GK;

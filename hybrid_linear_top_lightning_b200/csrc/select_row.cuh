@@ -3,17 +3,22 @@
 // the M highest summed scores are kept).  Order (score desc, position asc);
 // positions are emitted by rank, i.e. in ascending position order.
 //
-// Radix select on the 32-bit order-preserving key of each score:
+// Radix select on the 32-bit order-preserving key of each score, with every
+// thread working on its own contiguous chunk of 64 positions per round of
+// kSelThreads * 64 positions (no warp walks a range serially):
 //  1. first digit = key bits [31:20] (4096 bins), from a histogram given by the
 //     caller (built while the scores were produced) or computed here;
-//  2. one ordered pass over the row: keys whose first digit is above the
-//     threshold digit are selected; keys equal to it are candidates, appended
-//     to per-warp lists in position order;
-//  3. two 10-bit refinements over the candidates only (or over the whole row
-//     when a warp's candidate list overflows);
-//  4. every warp knows how many of its positions are selected (ties at the
-//     threshold key go to the lowest positions); warps whose rank range meets
-//     [lo, hi) walk their positions and write out[rank - lo] = position.
+//  2. the keys whose first digit equals the threshold digit are the
+//     candidates: counted per thread, then written in position order at
+//     block-scanned offsets;
+//  3. two 10-bit refinements over the candidates (or over the whole row when
+//     there are more than the candidate buffer holds) give the exact M-th
+//     largest key tau and how many keys equal to tau are kept;
+//  4. per thread, bit masks of its keys above tau and equal to tau; a block
+//     scan of the tie counts gives each tie its rank in position order (ties
+//     go to the lowest positions), a block scan of the selected counts gives
+//     each selected position its rank; positions whose rank falls in
+//     [lo, hi) are written to out[rank - lo].
 #pragma once
 
 #include "lisa_internal.cuh"
@@ -22,12 +27,15 @@ namespace lisa {
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kCandCap = 256;  // candidates per warp kept in shared memory
+constexpr int kCandCap = 256;                         // candidate slots per warp
+constexpr int kCandTotal = kSelWarps * kCandCap;      // candidate buffer (entries)
+constexpr int kSelChunk = 64;                         // positions per thread per round
+constexpr int kSelRound = kSelThreads * kSelChunk;    // positions per round
 
 struct SelectSmem {
     unsigned* hist;   // 4096 u32
-    int* bc;          // >= 64 ints: broadcasts and per-warp counts
-    uint2* cand;      // kSelWarps * kCandCap (key, position)
+    int* bc;          // >= 64 ints: broadcasts and scan scratch
+    uint2* cand;      // kCandTotal (key, position)
 };
 
 __device__ __forceinline__ int sel_block_excl_scan(int v, int* scratch, int& total) {
@@ -78,35 +86,37 @@ __device__ __forceinline__ void sel_find_bin(const unsigned* hv, int bpt, int ne
     __syncthreads();
 }
 
-// row: n scores, resident in shared memory (`resident`) or in global memory
-// (read through L2); the row buffer holds at least round_up(n, 8) floats.
-// M < n.  first_hist: 4096-bin histogram of key >> 20 over the row, or null.
-// row_bar: if not null, an mbarrier (phase 0) that completes when a TMA copy
-// of the row into shared memory has landed; it is waited on (bounded) after
-// the first digit is known, so the copy overlaps the histogram work.
+// Keeps the `keep` lowest set bits of m.
+__device__ __forceinline__ uint64_t sel_lowest_bits(uint64_t m, int keep) {
+    uint64_t r = 0;
+    for (int i = 0; i < keep && m; ++i) {
+        const uint64_t b = m & (~m + 1);
+        r |= b;
+        m ^= b;
+    }
+    return r;
+}
+
+// row: n scores, resident in shared memory (`resident`) or in global memory;
+// the row buffer holds at least round_up(n, 4) floats.  M < n.  first_hist:
+// 4096-bin histogram of key >> 20 over the row, or null.  row_bar: if not
+// null, an mbarrier (phase 0) that completes when a TMA copy of the row into
+// shared memory has landed; it is waited on (bounded) before the row is read,
+// after the first digit when that comes from first_hist.
 static __device__ void row_topm(const float* row, bool resident, int n, int M, const unsigned* first_hist,
-                         const SelectSmem& sm, int lo, int hi, int* out, uint64_t* row_bar,
-                         unsigned* status) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    auto keys8 = [&](int base, uint32_t (&k)[8]) {
-        const float4* src = reinterpret_cast<const float4*>(row) + base / 4;
-        float4 v0, v1;
-        if (resident) { v0 = src[0]; v1 = src[1]; }
-        else { v0 = __ldcg(src); v1 = __ldcg(src + 1); }
-        k[0] = order_key(v0.x); k[1] = order_key(v0.y); k[2] = order_key(v0.z); k[3] = order_key(v0.w);
-        k[4] = order_key(v1.x); k[5] = order_key(v1.y); k[6] = order_key(v1.z); k[7] = order_key(v1.w);
-    };
-    auto warp_excl = [&](int v, int& tot) {
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        tot = __shfl_sync(0xffffffffu, incl, 31);
-        return incl - v;
-    };
+                                const SelectSmem& sm, int lo, int hi, int* out, uint64_t* row_bar,
+                                unsigned* status) {
+    const int tid = threadIdx.x;
     int* bc = sm.bc;
+    const int rounds = (n + kSelRound - 1) / kSelRound;
+    // float4 j (0..15) of this thread's chunk in round r, visited in a rotated
+    // order so that the lanes of a quarter warp hit distinct shared-memory banks
+    auto chunk_q = [&](int r, int j) { return (r * kSelRound + tid * kSelChunk) / 4 + ((j + tid) & 15); };
+    auto load4 = [&](int q, uint32_t (&k)[4]) {
+        const float4* src = reinterpret_cast<const float4*>(row) + q;
+        const float4 v = resident ? *src : __ldg(src);
+        k[0] = order_key(v.x); k[1] = order_key(v.y); k[2] = order_key(v.z); k[3] = order_key(v.w);
+    };
     auto wait_row = [&]() {
         if (!row_bar) return;
         bool ok = false;
@@ -125,6 +135,7 @@ static __device__ void row_topm(const float* row, bool resident, int n, int M, c
         // works on stale shared memory, and the status word says so
         if (!ok && tid == 0) record_error(status, kDevTimeout);
     };
+
     // ---- 1. first digit
     uint32_t b1;
     int krem;
@@ -141,13 +152,17 @@ static __device__ void row_topm(const float* row, bool resident, int n, int M, c
             wait_row();
             for (int i = tid; i < 4096; i += kSelThreads) sm.hist[i] = 0u;
             __syncthreads();
-            for (int i8 = tid * 8; i8 < n; i8 += kSelThreads * 8) {
-                uint32_t k[8];
-                keys8(i8, k);
+            for (int r = 0; r < rounds; ++r)
+#pragma unroll 4
+                for (int j = 0; j < 16; ++j) {
+                    const int q = chunk_q(r, j);
+                    if (4 * q >= n) continue;
+                    uint32_t k[4];
+                    load4(q, k);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (i8 + e < n) atomicAdd(&sm.hist[k[e] >> 20], 1u);
-            }
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * q + e < n) atomicAdd(&sm.hist[k[e] >> 20], 1u);
+                }
             __syncthreads();
 #pragma unroll
             for (int q = 0; q < 16; ++q) hv[q] = sm.hist[tid * 16 + q];
@@ -157,46 +172,39 @@ static __device__ void row_topm(const float* row, bool resident, int n, int M, c
         krem = bc[1];
     }
     if (first_hist) wait_row();
-    // ---- 2. ordered candidate pass.  Warp w owns positions [w*seg, (w+1)*seg),
-    // walked in blocks of 256 with lane l on positions blk + 8l .. blk + 8l + 7.
-    const int seg = ((n + kSelWarps - 1) / kSelWarps + 255) / 256 * 256;
-    const int s0 = warp * seg, s1 = min(n, s0 + seg);
-    uint2* clist = sm.cand + warp * kCandCap;
-    int n_above = 0, ncand = 0;
-#pragma unroll 1
-    for (int blk = s0; blk < s1; blk += 256) {
-        const int base = blk + lane * 8;
-        uint32_t k[8];
-        unsigned cm = 0;
-        if (base < s1) {
-            keys8(base, k);
+
+    // ---- 2. candidates (first digit == b1), in position order
+    int ncand;
+    {
+        int mine = 0;
+        for (int r = 0; r < rounds; ++r)
+#pragma unroll 4
+            for (int j = 0; j < 16; ++j) {
+                const int q = chunk_q(r, j);
+                if (4 * q >= n) continue;
+                uint32_t k[4];
+                load4(q, k);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const bool v = base + e < s1;
-                n_above += v && (k[e] >> 20) > b1;
-                cm |= (unsigned)(v && (k[e] >> 20) == b1) << e;
+                for (int e = 0; e < 4; ++e) mine += (4 * q + e < n) && (k[e] >> 20) == b1;
             }
+        int off = sel_block_excl_scan(mine, bc + 32, ncand);
+        if (ncand <= kCandTotal && mine > 0) {
+            for (int r = 0; r < rounds; ++r)
+                for (int j = 0; j < 16; ++j) {
+                    const int q = (r * kSelRound + tid * kSelChunk) / 4 + j;  // position order
+                    if (4 * q >= n) continue;
+                    uint32_t k[4];
+                    load4(q, k);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if ((4 * q + e < n) && (k[e] >> 20) == b1)
+                            sm.cand[off++] = make_uint2(k[e], (uint32_t)(4 * q + e));
+                }
         }
-        int ctot;
-        int w = ncand + warp_excl(__popc(cm), ctot);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if ((cm >> e) & 1u) {
-                if (w < kCandCap) clist[w] = make_uint2(k[e], (uint32_t)(base + e));
-                ++w;
-            }
-        ncand += ctot;
+        __syncthreads();
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, o);
-    int* above_w = bc + 8;   // [kSelWarps]
-    int* ncand_w = bc + 16;  // [kSelWarps]
-    int* gt_w = bc + 24;     // [kSelWarps]
-    int* eq_w = bc + 48;     // [kSelWarps]  (bc + 32 .. 39 is the scan scratch)
-    if (lane == 0) { above_w[warp] = n_above; ncand_w[warp] = ncand; }
-    __syncthreads();
-    bool overflow = false;
-    for (int w = 0; w < kSelWarps; ++w) overflow |= ncand_w[w] > kCandCap;
+    const bool overflow = ncand > kCandTotal;
+
     // ---- 3. refinements
     uint32_t prefix = b1 << 20, mask = 0xFFFu << 20;
 #pragma unroll 1
@@ -205,22 +213,22 @@ static __device__ void row_topm(const float* row, bool resident, int n, int M, c
         for (int i = tid; i < 1024; i += kSelThreads) sm.hist[i] = 0u;
         __syncthreads();
         if (!overflow) {
-            for (int i = tid; i < kSelWarps * kCandCap; i += kSelThreads) {
-                const int w = i / kCandCap, c = i % kCandCap;
-                if (c < ncand_w[w]) {
-                    const uint32_t k = sm.cand[i].x;
-                    if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 1023u], 1u);
-                }
+            for (int i = tid; i < ncand; i += kSelThreads) {
+                const uint32_t k = sm.cand[i].x;
+                if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> shift) & 1023u], 1u);
             }
         } else {
-            for (int i8 = tid * 8; i8 < n; i8 += kSelThreads * 8) {
-                uint32_t k[8];
-                keys8(i8, k);
+            for (int r = 0; r < rounds; ++r)
+                for (int j = 0; j < 16; ++j) {
+                    const int q = chunk_q(r, j);
+                    if (4 * q >= n) continue;
+                    uint32_t k[4];
+                    load4(q, k);
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (i8 + e < n && (k[e] & mask) == prefix)
-                        atomicAdd(&sm.hist[(k[e] >> shift) & 1023u], 1u);
-            }
+                    for (int e = 0; e < 4; ++e)
+                        if (4 * q + e < n && (k[e] & mask) == prefix)
+                            atomicAdd(&sm.hist[(k[e] >> shift) & 1023u], 1u);
+                }
         }
         __syncthreads();
         unsigned hv[4];
@@ -230,75 +238,47 @@ static __device__ void row_topm(const float* row, bool resident, int n, int M, c
         prefix |= (uint32_t)bc[0] << shift;
         krem = bc[1];
         mask |= 1023u << shift;
-        __syncthreads();
     }
     const uint32_t tau = prefix;  // the M-th largest key; krem of its ties are kept
-    // ---- 4. per-warp selected counts, then the ranked walk
-    int gt_c = 0, eq_c = 0;
-    if (!overflow) {
-        for (int c = lane; c < ncand_w[warp]; c += 32) {
-            const uint32_t k = clist[c].x;
-            gt_c += k > tau;
-            eq_c += k == tau;
-        }
-    } else {
-        for (int blk = s0; blk < s1; blk += 256) {
-            const int base = blk + lane * 8;
-            if (base >= s1) continue;
-            uint32_t k[8];
-            keys8(base, k);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (base + e < s1 && (k[e] >> 20) == b1) { gt_c += k[e] > tau; eq_c += k[e] == tau; }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        gt_c += __shfl_xor_sync(0xffffffffu, gt_c, o);
-        eq_c += __shfl_xor_sync(0xffffffffu, eq_c, o);
-    }
-    if (lane == 0) { gt_w[warp] = gt_c; eq_w[warp] = eq_c; }
-    __syncthreads();
-    int eq_before = 0, sel_before = 0;
-    for (int w = 0; w < warp; ++w) {
-        const int eqw = eq_w[w];
-        sel_before += above_w[w] + gt_w[w] + max(0, min(eqw, krem - eq_before));
-        eq_before += eqw;
-    }
-    const int sel_mine = n_above + gt_c + max(0, min(eq_c, krem - eq_before));
-    if (sel_before < hi && sel_before + sel_mine > lo) {
+
+    // ---- 4. ranks in position order, round by round
+    int rank_base = 0, tie_base = 0;
 #pragma unroll 1
-        for (int blk = s0; blk < s1; blk += 256) {
-            const int base = blk + lane * 8;
-            uint32_t k[8];
-            unsigned eqm = 0, selm = 0;
-            if (base < s1) {
-                keys8(base, k);
+    for (int r = 0; r < rounds && rank_base < hi; ++r) {
+        uint64_t gtm = 0, eqm = 0;
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+            const int q = chunk_q(r, j);
+            if (4 * q >= n) continue;
+            uint32_t k[4];
+            load4(q, k);
+            const int bit = ((j + tid) & 15) * 4;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const bool v = base + e < s1;
-                    const bool above = v && (k[e] >> 20) > b1;
-                    const bool cand = v && (k[e] >> 20) == b1;
-                    eqm |= (unsigned)(cand && k[e] == tau) << e;
-                    selm |= (unsigned)(above || (cand && k[e] > tau)) << e;
-                }
+            for (int e = 0; e < 4; ++e) {
+                const bool v = 4 * q + e < n;
+                gtm |= (uint64_t)(v && k[e] > tau) << (bit + e);
+                eqm |= (uint64_t)(v && k[e] == tau) << (bit + e);
             }
-            int eq_tot;
-            int er = eq_before + warp_excl(__popc(eqm), eq_tot);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if ((eqm >> e) & 1u) { selm |= (unsigned)(er < krem) << e; ++er; }
-            int sel_tot;
-            int rank = sel_before + warp_excl(__popc(selm), sel_tot);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if ((selm >> e) & 1u) {
-                    if (rank >= lo && rank < hi) out[rank - lo] = base + e;
-                    ++rank;
-                }
-            eq_before += eq_tot;
-            sel_before += sel_tot;
-            if (sel_before >= hi) break;  // warp-uniform
+        }
+        const int eq_t = __popcll(eqm);
+        int eq_tot;
+        const int tie_before = tie_base + sel_block_excl_scan(eq_t, bc + 32, eq_tot);
+        tie_base += eq_tot;
+        const int keep = max(0, min(eq_t, krem - tie_before));
+        const uint64_t selm = gtm | sel_lowest_bits(eqm, keep);
+        const int sel_t = __popcll(selm);
+        int sel_tot;
+        int rank = rank_base + sel_block_excl_scan(sel_t, bc + 32, sel_tot);
+        rank_base += sel_tot;
+        if (rank < hi && rank + sel_t > lo) {
+            const int pos0 = r * kSelRound + tid * kSelChunk;
+            uint64_t m = selm;
+            while (m) {
+                const int b = __ffsll((long long)m) - 1;
+                m &= m - 1;
+                if (rank >= lo && rank < hi) out[rank - lo] = pos0 + b;
+                ++rank;
+            }
         }
     }
     __syncthreads();
