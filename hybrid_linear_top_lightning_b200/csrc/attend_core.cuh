@@ -14,7 +14,8 @@
 // probabilities are transposed in registers (movmatrix) and O^T[dim][head] +=
 // V^T[dim][key] P^T[key][head].  The warps serving one KV head split each
 // stage's keys 16 apiece and keep their own online-softmax state (base 2);
-// attn_core merges them at the end.
+// at the end the first warp of each KV head merges the others' states into
+// its registers (one exchange through shared memory).
 #pragma once
 
 #include "lisa_internal.cuh"
@@ -38,41 +39,62 @@ struct AttGeo {
     static constexpr int cpt = 2 * rpc / tpk;             // chunks per copying thread
     static constexpr int stage_bytes = keys * 2 * krow;   // K rows, then V rows
     static constexpr int ring_bytes = kAttStages * stage_bytes;
-    // merge scratch (in the ring after the loop): per warp O^T [8][128] + m[8] + l[8]
-    static constexpr int part_floats = 8 * d + 16;
-    static constexpr int res_off = kAttWarps * part_floats * 4;
-    // merged result: o [HKV*8][128], m [HKV*8], l [HKV*8] (floats)
-    static constexpr int res_bytes = (HKV * 8 * d + 2 * HKV * 8) * 4;
+    // merge exchange (in the ring after the loop): per warp 36 floats per lane
+    static constexpr int xfer_bytes = kAttWarps * 36 * 32 * 4;
     static_assert(cpt * tpk == 2 * rpc, "chunk split");
-    static_assert(res_off + res_bytes <= ring_bytes, "merge scratch fits in the ring");
+    static_assert(xfer_bytes <= ring_bytes, "merge exchange fits in the ring");
 };
 
-// Merged result of attn_core, in shared memory (inside the ring): for KV head
-// g and head slot r of its group (r < 8), the base-2 running max m, the sum l
-// and the un-normalised output o[0..128) relative to m.
-struct AttResult {
-    const float* o;  // [(g * 8 + r) * 128 + dim]
-    const float* m;  // [g * 8 + r]
-    const float* l;  // [g * 8 + r]
+// Query fragments of one row (B operand of the score MMA): per thread, head
+// gid of the warp's KV-head group, dims ks*16 + 2tq (+1) and + 8 (+9); heads
+// past the group are zero.  Loaded before the positions are known.
+struct AttQ {
+    uint32_t f[8][2];
 };
 
-// q_row: [H_q][128] bf16 (global) of this query row, `group` <= 8 heads per
-// KV head.  pos[0..cnt): positions (shared or global memory).  Position
+template <int HKV>
+__device__ __forceinline__ AttQ attn_load_q(const __nv_bfloat16* q_row, int group) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gid = lane >> 2, tq = lane & 3;
+    const int g_w = warp / AttGeo<HKV>::wph;
+    const bool live = gid < group;
+    const uint32_t* qh =
+        reinterpret_cast<const uint32_t*>(q_row + (int64_t)(g_w * group + (live ? gid : 0)) * 128);
+    AttQ q;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        q.f[ks][0] = live ? __ldg(qh + ks * 8 + tq) : 0u;
+        q.f[ks][1] = live ? __ldg(qh + ks * 8 + 4 + tq) : 0u;
+    }
+    return q;
+}
+
+// Online-softmax state of one KV head's query heads, held by the first warp
+// (part 0) of the head after attn_core: lane (gid, tq) has head slots
+// r = 2tq + h (h = 0, 1) with base-2 running max m[h] and sum l[h], and the
+// un-normalised output o[t][e] of slot 2tq + (e & 1), dim t*16 + gid + 8*(e >> 1).
+struct AttOut {
+    float m[2];
+    float l[2];
+    float o[8][4];
+};
+
+// q: the row's query fragments (attn_load_q), `group` <= 8 heads per KV
+// head.  pos[0..cnt): positions (shared or global memory).  Position
 // `p_special` (if >= 0) is read from k_special / v_special instead of the
 // caches.  Positions outside [0, p_max] are masked out and reported through
 // `status`.  `ring` holds AttGeo<HKV>::ring_bytes bytes, `spos` (shared
-// memory) kAttStages * AttGeo<HKV>::keys ints.  Ends with a block barrier;
-// the result stays valid until the ring is reused.
+// memory) kAttStages * AttGeo<HKV>::keys ints; both are clobbered.  The
+// result is valid in the warps with part == 0 (warp % wph == 0).
 template <int HKV>
-__device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int group, uint8_t* ring,
-                                               int* spos, const int* pos, int cnt,
-                                               const __nv_bfloat16* k_cache,
-                                               const __nv_bfloat16* v_cache,
-                                               int64_t row0,  // b * N_max
-                                               int p_max, int p_special,
-                                               const __nv_bfloat16* k_special,
-                                               const __nv_bfloat16* v_special, float scale_log2,
-                                               unsigned* status) {
+__device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spos, const int* pos,
+                                          int cnt, const __nv_bfloat16* k_cache,
+                                          const __nv_bfloat16* v_cache,
+                                          int64_t row0,  // b * N_max
+                                          int p_max, int p_special,
+                                          const __nv_bfloat16* k_special,
+                                          const __nv_bfloat16* v_special, float scale_log2,
+                                          unsigned* status, AttOut& out) {
     using A = AttGeo<HKV>;
     using bf16 = __nv_bfloat16;
     constexpr int GK = A::keys;
@@ -82,20 +104,6 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
     const int key0 = part * 16;  // this warp's keys within a stage
     const int nst = (cnt + GK - 1) / GK;
     constexpr int kb_row = HKV * 128;
-
-    // query fragments (B operand of the score MMA): head gid of group g_w,
-    // dims ks*16 + 2tq (+1) and + 8 (+9); heads past the group are zero
-    uint32_t qf[8][2];
-    {
-        const bool live = gid < group;
-        const uint32_t* qh =
-            reinterpret_cast<const uint32_t*>(q_row + (int64_t)(g_w * group + (live ? gid : 0)) * 128);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qf[ks][0] = live ? __ldg(qh + ks * 8 + tq) : 0u;
-            qf[ks][1] = live ? __ldg(qh + ks * 8 + 4 + tq) : 0u;
-        }
-    }
 
     // copy role: thread copies chunks sub, sub + tpk, ... of key ck's K and V rows
     const int ck = tid / A::tpk, sub = tid % A::tpk;
@@ -121,9 +129,11 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
         }
     };
 
-    float m[2] = {-INFINITY, -INFINITY};  // heads 2tq, 2tq + 1
-    float l[2] = {0.0f, 0.0f};
-    float o[8][4];
+    float* m = out.m;  // heads 2tq, 2tq + 1
+    float* l = out.l;
+    float (*o)[4] = out.o;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.0f;
 #pragma unroll
     for (int t = 0; t < 8; ++t)
 #pragma unroll
@@ -162,8 +172,8 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
             uint32_t a0[4], a1[4];
             ptx::ldmatrix_x4(a0, kb + ka_key * A::krow + head_off + (ks * 16 + ka_dim) * 2);
             ptx::ldmatrix_x4(a1, kb + ka_key * A::krow + head_off + ((ks + 1) * 16 + ka_dim) * 2);
-            ptx::mma_bf16(s0, a0, qf[ks][0], qf[ks][1]);
-            ptx::mma_bf16(s1, a1, qf[ks + 1][0], qf[ks + 1][1]);
+            ptx::mma_bf16(s0, a0, q.f[ks][0], q.f[ks][1]);
+            ptx::mma_bf16(s1, a1, q.f[ks + 1][0], q.f[ks + 1][1]);
         }
         // element e: key key0 + gid + 8 (e >> 1), head 2tq + (e & 1)
         float v[4];
@@ -220,53 +230,37 @@ __device__ __forceinline__ AttResult attn_core(const __nv_bfloat16* q_row, int g
         l[h] += __shfl_xor_sync(0xffffffffu, l[h], 8);
         l[h] += __shfl_xor_sync(0xffffffffu, l[h], 16);
     }
+    if (A::wph == 1) return;
     __syncthreads();  // every warp is done with the ring
 
-    // ---- merge the warps of each KV head
-    float* ringf = reinterpret_cast<float*>(ring);
-    float* pw = ringf + warp * A::part_floats;
+    // ---- the other warps of the KV head hand their state to its first warp
+    float* xf = reinterpret_cast<float*>(ring) + warp * 36 * 32 + lane;  // [36][32] per warp
+    if (part != 0) {
+        xf[0] = m[0]; xf[32] = m[1]; xf[64] = l[0]; xf[96] = l[1];
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < 8; ++t)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            pw[(2 * tq + (e & 1)) * 128 + t * 16 + gid + 8 * (e >> 1)] = o[t][e];
-    if (gid == 0) {
-        pw[8 * 128 + 2 * tq] = m[0];
-        pw[8 * 128 + 2 * tq + 1] = m[1];
-        pw[8 * 128 + 8 + 2 * tq] = l[0];
-        pw[8 * 128 + 8 + 2 * tq + 1] = l[1];
+            for (int e = 0; e < 4; ++e) xf[(4 + t * 4 + e) * 32] = o[t][e];
     }
     __syncthreads();
-    float* res = reinterpret_cast<float*>(ring + A::res_off);
-    float* res_m = res + HKV * 8 * 128;
-    float* res_l = res_m + HKV * 8;
-    for (int e = tid; e < HKV * 8 * 128; e += kAttThreads) {
-        const int hs = e / 128, dim = e % 128;  // hs = g * 8 + r
-        const int g = hs / 8, r = hs % 8;
-        float M = -INFINITY;
+    if (part != 0) return;
+#pragma unroll 1
+    for (int k = 1; k < A::wph; ++k) {
+        const float* yf = xf + k * 36 * 32;
 #pragma unroll
-        for (int k = 0; k < A::wph; ++k)
-            M = fmaxf(M, ringf[(g * A::wph + k) * A::part_floats + 8 * 128 + r]);
-        float L = 0.0f, O = 0.0f;
-        if (M != -INFINITY) {
+        for (int h = 0; h < 2; ++h) {
+            const float mk = yf[h * 32], lk = yf[(2 + h) * 32];
+            const float M = fmaxf(m[h], mk);
+            const float a = (m[h] == -INFINITY) ? 0.0f : exp2f(m[h] - M);
+            const float c = (mk == -INFINITY) ? 0.0f : exp2f(mk - M);
+            m[h] = M;
+            l[h] = l[h] * a + lk * c;
 #pragma unroll
-            for (int k = 0; k < A::wph; ++k) {
-                const float* q = ringf + (g * A::wph + k) * A::part_floats;
-                const float mk = q[8 * 128 + r];
-                if (mk == -INFINITY) continue;
-                const float w = exp2f(mk - M);
-                L = fmaf(q[8 * 128 + 8 + r], w, L);
-                O = fmaf(q[r * 128 + dim], w, O);
-            }
-        }
-        res[e] = O;
-        if (dim == 0) {
-            res_m[hs] = M;
-            res_l[hs] = L;
+            for (int t = 0; t < 8; ++t)
+#pragma unroll
+                for (int e = h; e < 4; e += 2) o[t][e] = o[t][e] * a + yf[(4 + t * 4 + e) * 32] * c;
         }
     }
-    __syncthreads();
-    return AttResult{res, res_m, res_l};
 }
 
 }  // namespace lisa

@@ -57,7 +57,6 @@ constexpr int kScanRows = 128;        // keys per TMA box (16 per warp)
 constexpr int kScanStages = 8;        // boxes in flight per CTA
 constexpr int kBoxBytes = kScanRows * kDI * 2;
 constexpr int kLaCols = 32;           // linear-state columns per slice
-constexpr int kMaxPer = 2048;         // selected positions per attend CTA
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
@@ -85,7 +84,8 @@ struct Params {
     bf16* o;
     int32_t* idx;
     int32_t* count;
-    float* scores;      // workspace [B][ns]
+    int32_t* sel;       // [B][M] selected positions: idx, or the workspace copy
+    uint32_t* keys;     // workspace [B][ns]: order-preserving keys of the scores
     float* olin;        // workspace [B][H_q][kD]
     float* part;        // workspace [B][S2][H_q][kD + 2]
     unsigned* hist;     // workspace [B][4096]: histogram of the top 12 bits of the score keys
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (2 * tq < P.H_I) w_lo = wb[2 * tq];
         if (2 * tq + 1 < P.H_I) w_hi = wb[2 * tq + 1];
     }
-    float* srow = P.scores + (int64_t)b * P.ns;
+    uint32_t* srow = P.keys + (int64_t)b * P.ns;
     for (int st = 0; st < nst; ++st) {
         const int buf = st % kScanStages;
         if (ok && !ptx::mbar_wait_bounded(&bars[buf], (st / kScanStages) & 1, kWaitTries)) {
@@ -358,9 +358,9 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (ok && tid < kScanRows) {
             const int pos = k0 + st * kScanRows + tid;
             if (pos < k1) {
-                const float v = ssc[tid];
-                srow[pos] = v;
-                atomicAdd(&lhist[order_key(v) >> 20], 1u);
+                const uint32_t kk = order_key(ssc[tid]);
+                srow[pos] = kk;
+                atomicAdd(&lhist[kk >> 20], 1u);
             }
         }
     }
@@ -378,24 +378,70 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     }
 }
 
-// ============================================================================ K2: attend
+// ============================================================================ K2: select
+// One CTA of kSelNT threads per sequence: the exact top-M of the score row
+// (row_topm), written once to the sequence's index row for the attend CTAs.
+constexpr int kSelNT = 1024;
+constexpr int kSelKeyCap = 40960;  // score keys of a row held in shared memory
+
+struct SelSmem {
+    static constexpr int hist = 0;                         // u32[4096]
+    static constexpr int cand = hist + 4096 * 4;           // uint2[kCandTotal]
+    static constexpr int bc = cand + kCandTotal * 8;       // int[64]
+    static constexpr int bar = bc + 64 * 4;                // mbarrier
+    static constexpr int row = bar + 128;                  // u32[kSelKeyCap]
+    static constexpr int total = row + kSelKeyCap * 4;
+    static_assert(total <= 227 * 1024, "shared memory per CTA");
+};
+
+__global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
+    extern __shared__ __align__(128) uint8_t sel_raw[];
+    uint64_t* rowbar = reinterpret_cast<uint64_t*>(sel_raw + SelSmem::bar);
+    uint32_t* row_smem = reinterpret_cast<uint32_t*>(sel_raw + SelSmem::row);
+    const int tid = threadIdx.x, b = blockIdx.x;
+    const int n = P.n;
+    ptx::pdl_launch_dependents();
+    if (tid == 0) {
+        ptx::mbar_init(rowbar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    ptx::pdl_wait_prior();  // score keys and histogram of this call are ready
+    int32_t* out = P.sel + (int64_t)b * P.M;
+    const int cnt = min(P.M, n);
+    if (tid == 0 && P.count) P.count[b] = cnt;
+    if (n <= P.M) {
+        for (int i = tid; i < P.M; i += kSelNT) out[i] = i < n ? i : -1;
+        return;
+    }
+    // Radix select on the order-preserving score keys, most significant digit
+    // first: 12 bits (the histogram the scan kernel built), then 10 and 10 bits
+    // over the keys that share the digits found so far.  Ties at the M-th key
+    // keep the lowest positions.
+    const uint32_t* srow = P.keys + (int64_t)b * P.ns;
+    const bool resident = n <= kSelKeyCap;
+    if (resident && tid == 0) {
+        const int bytes = ((n + 3) / 4) * 16;
+        ptx::mbar_arrive_expect_tx(rowbar, bytes);
+        for (int off = 0; off < bytes; off += 16384)
+            ptx::bulk_load(reinterpret_cast<uint8_t*>(row_smem) + off, srow + off / 4,
+                           min(16384, bytes - off), rowbar);
+    }
+    SelectSmem sel;
+    sel.hist = reinterpret_cast<unsigned*>(sel_raw + SelSmem::hist);
+    sel.bc = reinterpret_cast<int*>(sel_raw + SelSmem::bc);
+    sel.cand = reinterpret_cast<uint2*>(sel_raw + SelSmem::cand);
+    row_topm<kSelNT>(resident ? row_smem : srow, resident, n, P.M, P.hist + (int64_t)b * 4096, sel,
+                     0, P.M, out, resident ? rowbar : nullptr, P.status);
+}
+
+// ============================================================================ K3: attend
 template <int HKV>
 struct Att : AttGeo<HKV> {
     using G = AttGeo<HKV>;
-    // shared memory: the gather ring first, which during selection holds the
-    // histogram, the candidate lists and (when it fits) the score row; then
-    // the barrier, broadcasts, selected positions and stage positions
-    static constexpr int ring = 0;
-    static constexpr int hist = ring;                                  // u32[4096]
-    static constexpr int cand = hist + 4096 * 4;                       // uint2[8][kCandCap]
-    static constexpr int row = cand + kAttWarps * kCandCap * 8;        // float[key_cap]
-    static constexpr int key_cap = (G::ring_bytes - row) / 4 - 32;     // scores that fit
-    static constexpr int bar = ring + G::ring_bytes;
-    static constexpr int bc = bar + 16;                                // int[128]
-    static constexpr int mypos = bc + 128 * 4;
-    static constexpr int spos = mypos + kMaxPer * 4;                   // int[stages][keys]
-    static constexpr int total = spos + kAttStages * G::keys * 4;
-    static_assert(row < G::ring_bytes, "selection scratch must fit in the gather ring");
+    static constexpr int spos = 0;                                     // int[stages][keys]
+    static constexpr int ring = (kAttStages * G::keys * 4 + 127) / 128 * 128;
+    static constexpr int total = ring + G::ring_bytes;
     static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -403,85 +449,47 @@ template <int HKV>
 __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P) {
     using A = Att<HKV>;
     extern __shared__ __align__(128) uint8_t att_raw[];
-    unsigned* hist = reinterpret_cast<unsigned*>(att_raw + A::hist);
-    uint64_t* rowbar = reinterpret_cast<uint64_t*>(att_raw + A::bar);
-    int* bc = reinterpret_cast<int*>(att_raw + A::bc);
-    int* mypos = reinterpret_cast<int*>(att_raw + A::mypos);
-    uint8_t* stage = att_raw + A::ring;
-    float* row_smem = reinterpret_cast<float*>(att_raw + A::row);
     int* spos = reinterpret_cast<int*>(att_raw + A::spos);
-
     const int tid = threadIdx.x;
     const int b = blockIdx.x / P.S2, j = blockIdx.x % P.S2;
     const int n = P.n, p = n - 1;
     ptx::pdl_launch_dependents();
-
-    // ---- prologue (inputs only; nothing written by the scan kernel)
-    if (tid == 0) {
-        ptx::mbar_init(rowbar, 1);
-        ptx::fence_mbar_init();
-    }
-    __syncthreads();
-    ptx::pdl_wait_prior();  // scores, histogram and linear output of this call are ready
-
-    // ---- exact top-M of the score row (the same result in every CTA of the sequence)
-    // Radix select on the 32-bit order-preserving key of each score, most
-    // significant digit first: 12 bits (the histogram the scan kernel built),
-    // then 10 and 10 bits over the keys that share the digits found so far.
-    // Ties at the M-th key keep the lowest positions.
-    const float* srow = P.scores + (int64_t)b * P.ns;
+    const AttQ q = attn_load_q<HKV>(P.q + (int64_t)b * P.H_q * kD, P.group);  // an input: before the wait
+    ptx::pdl_wait_prior();  // the index row of this sequence is complete
     const int cnt = min(P.M, n);
     const int lo = j * P.per, hi = min(cnt, lo + P.per);
     const int mine = max(0, hi - lo);
-    if (n <= P.M) {
-        for (int i = tid; i < mine; i += kAttThreads) mypos[i] = lo + i;
-    } else {
-        // the score row comes into shared memory by TMA bulk copies when it fits
-        const bool resident = n <= A::key_cap;
-        if (resident && tid == 0) {
-            const int bytes = ((n + 3) / 4) * 16;
-            ptx::mbar_arrive_expect_tx(rowbar, bytes);
-            for (int off = 0; off < bytes; off += 16384)
-                ptx::bulk_load(reinterpret_cast<uint8_t*>(row_smem) + off, srow + off / 4,
-                               min(16384, bytes - off), rowbar);
-        }
-        SelectSmem sel;
-        sel.hist = hist;
-        sel.bc = bc;
-        sel.cand = reinterpret_cast<uint2*>(att_raw + A::cand);
-        row_topm(resident ? row_smem : srow, resident, n, P.M,
-                 P.hist + (int64_t)b * 4096, sel, lo, hi, mypos, resident ? rowbar : nullptr,
-                 P.status);
-    }
-    __syncthreads();
-    if (P.idx) {
-        for (int i = tid; i < mine; i += kAttThreads) P.idx[(int64_t)b * P.M + lo + i] = mypos[i];
-        if (j == 0)
-            for (int i = cnt + tid; i < P.M; i += kAttThreads) P.idx[(int64_t)b * P.M + i] = -1;
-    }
-    if (P.count && j == 0 && tid == 0) P.count[b] = cnt;
 
-    // ---- gather + attention over this CTA's positions
+    // ---- gather + attention over this CTA's share of the selected positions
     constexpr int kb_row = HKV * kD;
-    const AttResult r = attn_core<HKV>(P.q + (int64_t)b * P.H_q * kD, P.group, stage, spos, mypos,
-                                       mine, P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p,
-                                       P.k_new + (int64_t)b * kb_row,
-                                       P.v_new + (int64_t)b * kb_row, P.scale_log2, P.status);
-    // partial (m, l, O) of this CTA for every query head
-    float* prow = P.part + ((int64_t)b * P.S2 + j) * P.H_q * (kD + 2);
-    for (int e = tid; e < P.H_q * kD; e += kAttThreads) {
-        const int h = e / kD, dim = e % kD;
-        const int hs = (h / P.group) * 8 + h % P.group;
-        float* rec = prow + (int64_t)h * (kD + 2);
-        rec[2 + dim] = r.o[hs * kD + dim];
-        if (dim == 0) {
-            rec[0] = r.m[hs];
-            rec[1] = r.l[hs];
+    AttOut r;
+    attn_core<HKV>(q, att_raw + A::ring, spos, P.sel + (int64_t)b * P.M + lo, mine, P.k_cache,
+                   P.v_cache, (int64_t)b * P.N_max, p, p, P.k_new + (int64_t)b * kb_row,
+                   P.v_new + (int64_t)b * kb_row, P.scale_log2, P.status, r);
+    // partial (m, l, O) of this CTA for every query head, from the first warp
+    // of each KV head
+    const int lane = tid & 31, warp = tid >> 5;
+    if (warp % AttGeo<HKV>::wph != 0) return;
+    const int g = warp / AttGeo<HKV>::wph, gid = lane >> 2, tq = lane & 3;
+    float* prow = P.part + (((int64_t)b * P.S2 + j) * P.H_q + g * P.group) * (kD + 2);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int slot = 2 * tq + h;
+        if (slot >= P.group) continue;
+        float* rec = prow + (int64_t)slot * (kD + 2);
+        if (gid == 0) {
+            rec[0] = r.m[h];
+            rec[1] = r.l[h];
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            rec[2 + t * 16 + gid] = r.o[t][h];
+            rec[2 + t * 16 + gid + 8] = r.o[t][h + 2];
         }
     }
 }
 
-// ============================================================================ K3: combine
+// ============================================================================ K4: combine
 // One CTA per (sequence, query head), one thread per output dimension: merge
 // the attend CTAs' partial (max, sum, output) triples, mix with the linear
 // branch through the gate, write o.  Also advances the elu+1 normaliser z and
@@ -547,7 +555,7 @@ int num_sms() {
 
 struct Plan {
     int S1, KPC, S2, per, ns;
-    size_t scores, olin, part, hist, end;
+    size_t scores, olin, part, hist, sel, end;
 };
 
 Plan make_plan(const Shape& s) {
@@ -568,10 +576,11 @@ Plan make_plan(const Shape& s) {
         off += (bytes + 255) & ~(size_t)255;
         return at;
     };
-    pl.scores = take(sizeof(float) * (size_t)s.B * pl.ns);
+    pl.scores = take(sizeof(uint32_t) * (size_t)s.B * pl.ns);
     pl.olin = take(sizeof(float) * (size_t)s.B * s.H_q * kD);
     pl.part = take(sizeof(float) * (size_t)s.B * pl.S2 * s.H_q * (kD + 2));
     pl.hist = take(sizeof(unsigned) * (size_t)s.B * 4096);
+    pl.sel = take(sizeof(int32_t) * (size_t)s.B * s.M);
     pl.end = off;
     return pl;
 }
@@ -589,8 +598,6 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
     if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD || s.d_I != kDI || s.H_Ik != 1) return false;
     if (s.H_I > 8 || s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
     if (s.L < 1 || s.M < 1 || s.B < 1) return false;
-    const Plan pl = make_plan(s);
-    if (pl.per > kMaxPer) return false;
     const void* ptrs[] = {a.q, a.k_new, a.v_new, a.q_I, a.k_I_new, a.q_L, a.k_L, a.v_L,
                           a.k_cache, a.v_cache, a.k_I_cache, a.S, a.o};
     for (const void* p : ptrs)
@@ -617,10 +624,11 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     P.S = a.S; P.z = a.z; P.o = (bf16*)a.o; P.idx = a.idx; P.count = a.count;
     char* w8 = (char*)ws;
     P.status = (unsigned*)ws;
-    P.scores = (float*)(w8 + pl.scores);
+    P.keys = (uint32_t*)(w8 + pl.scores);
     P.olin = (float*)(w8 + pl.olin);
     P.part = (float*)(w8 + pl.part);
     P.hist = (unsigned*)(w8 + pl.hist);
+    P.sel = a.idx ? a.idx : (int32_t*)(w8 + pl.sel);
 
     CUtensorMap tmap;
     if (!make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max, kScanRows))
@@ -632,6 +640,9 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     if (dev < 0 || dev >= 64 || !attrs_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(k_decode_scan, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              ScanSmem::total);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_decode_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SelSmem::total);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_decode_attend<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Att<1>::total);
@@ -657,6 +668,13 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.gridDim = dim3(s.B);
+    cfg.blockDim = dim3(kSelNT);
+    cfg.dynamicSmemBytes = SelSmem::total;
+    e = cudaLaunchKernelEx(&cfg, k_decode_select, P);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(s.B * pl.S2);
+    cfg.blockDim = dim3(kAttThreads);
     switch (s.H_kv) {
         case 1: cfg.dynamicSmemBytes = Att<1>::total; e = cudaLaunchKernelEx(&cfg, k_decode_attend<1>, P); break;
         case 2: cfg.dynamicSmemBytes = Att<2>::total; e = cudaLaunchKernelEx(&cfg, k_decode_attend<2>, P); break;

@@ -45,7 +45,7 @@ struct ScoreParams {
     int B, T, n_past, L, Lpad, N_max, H_I, nqt;
     int64_t w_tok_stride;
     const float* w;
-    float* scores;  // [B*T][Lpad]
+    uint32_t* keys;  // [B*T][Lpad]: order-preserving keys of the causal scores
     unsigned* status;
 };
 
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
                         sc = fmaf(ws[ql * 8 + h], fmaxf(__uint_as_float(r[u * HI + h]), 0.0f), sc);
                     const int t = q0 + ql;
                     if (ql < qrows && key < P.L && key <= P.n_past + t)
-                        P.scores[((int64_t)b * P.T + t) * P.Lpad + key] = sc;
+                        P.keys[((int64_t)b * P.T + t) * P.Lpad + key] = order_key(sc);
                 }
             }
             ptx::tc_fence_before();
@@ -214,10 +214,11 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
 
 // ---------------------------------------------------------------- per-row selection
 constexpr int kRowCap = 16384;  // scores of a row held in shared memory
+constexpr int kRowThreads = 256;
 
 struct RowParams {
     int B, T, n_past, Lpad, M;
-    const float* scores;
+    const uint32_t* keys;
     int32_t* idx;
     int32_t* count;
     unsigned* status;
@@ -226,13 +227,13 @@ struct RowParams {
 struct RowSmem {
     static constexpr int row = 0;                         // float[kRowCap + 32]
     static constexpr int hist = row + (kRowCap + 32) * 4; // u32[4096]
-    static constexpr int cand = hist + 4096 * 4;          // uint2[8][kCandCap]
-    static constexpr int bc = cand + kSelWarps * kCandCap * 8;
+    static constexpr int cand = hist + 4096 * 4;          // uint2[kCandTotal]
+    static constexpr int bc = cand + kCandTotal * 8;
     static constexpr int bar = bc + 128 * 4;
     static constexpr int total = bar + 16;
 };
 
-__global__ void __launch_bounds__(kSelThreads) k_topm_rows_fast(const RowParams P) {
+__global__ void __launch_bounds__(kRowThreads) k_topm_rows_fast(const RowParams P) {
     extern __shared__ __align__(128) uint8_t row_raw[];
     const int row = blockIdx.x;
     const int t = row % P.T;
@@ -240,13 +241,13 @@ __global__ void __launch_bounds__(kSelThreads) k_topm_rows_fast(const RowParams 
     int32_t* out = P.idx + (int64_t)row * P.M;
     ptx::pdl_wait_prior();
     if (nc <= P.M) {
-        for (int i = threadIdx.x; i < P.M; i += kSelThreads) out[i] = i < nc ? i : -1;
+        for (int i = threadIdx.x; i < P.M; i += kRowThreads) out[i] = i < nc ? i : -1;
         if (threadIdx.x == 0) P.count[row] = nc;
         return;
     }
-    float* rs = reinterpret_cast<float*>(row_raw + RowSmem::row);
+    uint32_t* rs = reinterpret_cast<uint32_t*>(row_raw + RowSmem::row);
     uint64_t* bar = reinterpret_cast<uint64_t*>(row_raw + RowSmem::bar);
-    const float* gr = P.scores + (int64_t)row * P.Lpad;
+    const uint32_t* gr = P.keys + (int64_t)row * P.Lpad;
     const bool resident = nc <= kRowCap;
     if (resident && threadIdx.x == 0) {
         ptx::mbar_init(bar, 1);
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topm_rows_fast(const RowParams 
     sel.hist = reinterpret_cast<unsigned*>(row_raw + RowSmem::hist);
     sel.bc = reinterpret_cast<int*>(row_raw + RowSmem::bc);
     sel.cand = reinterpret_cast<uint2*>(row_raw + RowSmem::cand);
-    row_topm(resident ? rs : gr, resident, nc, P.M, nullptr, sel, 0, P.M, out,
+    row_topm<kRowThreads>(resident ? rs : gr, resident, nc, P.M, nullptr, sel, 0, P.M, out,
              resident ? bar : nullptr, P.status);
     if (threadIdx.x == 0) P.count[row] = P.M;
 }
@@ -293,7 +294,7 @@ cudaError_t fast_topm(const Shape& s, const void* q_I, const void* k_I, const fl
     P.B = s.B; P.T = s.T; P.n_past = s.n_past; P.L = s.L; P.Lpad = (s.L + 31) / 32 * 32;
     P.N_max = s.N_max; P.H_I = s.H_I; P.nqt = (s.T + kQT - 1) / kQT;
     P.w_tok_stride = w_tok_stride; P.w = w;
-    P.scores = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kStatusBytes);
+    P.keys = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + kStatusBytes);
     P.status = reinterpret_cast<unsigned*>(ws);
     CUtensorMap tq, tk;
     const int N = kQT * s.H_I;
@@ -327,13 +328,13 @@ cudaError_t fast_topm(const Shape& s, const void* q_I, const void* k_I, const fl
     if (e != cudaSuccess) return e;
     RowParams R;
     R.B = s.B; R.T = s.T; R.n_past = s.n_past; R.Lpad = P.Lpad; R.M = s.M;
-    R.scores = P.scores; R.idx = idx; R.count = count; R.status = P.status;
+    R.keys = P.keys; R.idx = idx; R.count = count; R.status = P.status;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(s.B * s.T);
-    cfg.blockDim = dim3(kSelThreads);
+    cfg.blockDim = dim3(kRowThreads);
     cfg.dynamicSmemBytes = RowSmem::total;
     cfg.stream = st;
     cfg.attrs = attr;

@@ -42,18 +42,32 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_sparse_rows(const SpParams P
     const int p = P.n_past + t;
     const int cnt = max(0, min(P.count[row], P.M));
     const int* pos = P.idx + (int64_t)row * P.M;  // read through L1 by the gather
-    const AttResult r = attn_core<HKV>(P.q + (int64_t)row * P.H_q * 128, P.group, sp_raw + L::ring,
-                                       spos, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1,
-                                       nullptr, nullptr, P.scale_log2, P.status);
-    // normalised output, two dims per thread
-    for (int e = threadIdx.x; e < P.H_q * 64; e += kAttThreads) {
-        const int h = e / 64, dim = (e % 64) * 2;
-        const int hs = (h / P.group) * 8 + h % P.group;
-        const float lsum = r.l[hs];
-        const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-        *reinterpret_cast<__nv_bfloat162*>(P.o + ((int64_t)row * P.H_q + h) * 128 + dim) =
-            __floats2bfloat162_rn(r.o[hs * 128 + dim] * inv, r.o[hs * 128 + dim + 1] * inv);
+    const AttQ q = attn_load_q<HKV>(P.q + (int64_t)row * P.H_q * 128, P.group);
+    AttOut r;
+    attn_core<HKV>(q, sp_raw + L::ring, spos, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1,
+                   nullptr, nullptr, P.scale_log2, P.status, r);
+    // normalised output of each KV head's query heads (group rows of 128 dims,
+    // contiguous in o), staged by the head's first warp in its own slot of the
+    // ring and stored with 16-byte writes
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp % AttGeo<HKV>::wph != 0) return;
+    const int g = warp / AttGeo<HKV>::wph, gid = lane >> 2, tq = lane & 3;
+    bf16* stage = reinterpret_cast<bf16*>(sp_raw + L::ring) + warp * 36 * 32 * 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int slot = 2 * tq + h;
+        if (slot >= P.group) continue;
+        const float inv = r.l[h] > 0.0f ? 1.0f / r.l[h] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            stage[slot * 128 + t * 16 + gid] = __float2bfloat16_rn(r.o[t][h] * inv);
+            stage[slot * 128 + t * 16 + gid + 8] = __float2bfloat16_rn(r.o[t][h + 2] * inv);
+        }
     }
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(P.o + ((int64_t)row * P.H_q + g * P.group) * 128);
+    const uint4* src = reinterpret_cast<const uint4*>(stage);
+    for (int c = lane; c < P.group * 16; c += 32) dst[c] = src[c];
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
