@@ -115,8 +115,7 @@ struct ScanSmem {
     static constexpr int vcol = fq + 16 * kD * 4;                    // float[32]
     static constexpr int zloc = vcol + kLaCols * 4;                  // float[128]
     static constexpr int den = zloc + kD * 4;                        // float[16]
-    static constexpr int stage_sc = den + 16 * 4;                    // float[2][128]
-    static constexpr int lhist = stage_sc + 2 * kScanRows * 4;       // u32[4096]
+    static constexpr int lhist = den + 16 * 4;                       // u32[4096]
     static constexpr int bars = lhist + 4096 * 4;                    // uint64[kScanStages]
     static constexpr int total = bars + kScanStages * 8 + 1024;      // + base alignment slack
 };
@@ -159,6 +158,7 @@ __device__ void linear_slice(const Params& P, int b, int g, int c0, float* s_sli
             for (int x = 0; x < 8; ++x) fq[h * kD + 8 * c8 + x] = feat(P.phi, f[x]);
         }
     }
+    ptx::cp_async_wait_all();  // the state slice (when it was prefetched)
     group_sync(kLaBar, kLaThreads);
     const bool norm = P.phi == LISA_PHI_ELU1_NORM;
     float* Sg = P.S + ((int64_t)b * P.H_kv + g) * kD * kD;
@@ -187,10 +187,14 @@ __device__ void linear_slice(const Params& P, int b, int g, int c0, float* s_sli
     }
     for (int e = tid; e < P.group * kLaCols; e += kLaThreads) {
         const int h = e / kLaCols, c = e % kLaCols;
-        float acc = 0.0f;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
 #pragma unroll 8
-        for (int i = 0; i < kD; ++i) acc = fmaf(fq[h * kD + i], s_slice[i * kLaCols + c], acc);
-        P.olin[((int64_t)b * P.H_q + g * P.group + h) * kD + c0 + c] = norm ? acc / den[h] : acc;
+        for (int i = 0; i < kD; i += 4)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                acc[u] = fmaf(fq[h * kD + i + u], s_slice[(i + u) * kLaCols + c], acc[u]);
+        const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        P.olin[((int64_t)b * P.H_q + g * P.group + h) * kD + c0 + c] = norm ? sum / den[h] : sum;
     }
     group_sync(kLaBar, kLaThreads);
 }
@@ -207,7 +211,6 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     float* vcol = reinterpret_cast<float*>(base + ScanSmem::vcol);
     float* zloc = reinterpret_cast<float*>(base + ScanSmem::zloc);
     float* den = reinterpret_cast<float*>(base + ScanSmem::den);
-    float* stage_sc = reinterpret_cast<float*>(base + ScanSmem::stage_sc);
     unsigned* lhist = reinterpret_cast<unsigned*>(base + ScanSmem::lhist);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + ScanSmem::bars);
 
@@ -248,8 +251,6 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     __syncthreads();  // barriers initialised; from here the two warp groups run apart
     if (la_thread) {
         if (slice < P.la_slices) {
-            ptx::cp_async_wait_all();
-            group_sync(kLaBar, kLaThreads);
             const int lb = slice / slices_per_b, lg = (slice / (kD / kLaCols)) % P.H_kv;
             const int lc0 = (slice % (kD / kLaCols)) * kLaCols;
             linear_slice(P, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
@@ -304,23 +305,29 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (2 * tq < P.H_I) w_lo = wb[2 * tq];
         if (2 * tq + 1 < P.H_I) w_hi = wb[2 * tq + 1];
     }
+    group_sync(kScanBar, kScanThreads);  // the local histogram is cleared
+    // Warp w owns ring slot w: it scores boxes w, w + 8, ... by itself (8 row
+    // tiles of 16 keys each) and re-arms its slot, so no barrier joins the
+    // scan warps until the histogram is merged.
     uint32_t* srow = P.keys + (int64_t)b * P.ns;
-    for (int st = 0; st < nst; ++st) {
-        const int buf = st % kScanStages;
-        if (ok && !ptx::mbar_wait_bounded(&bars[buf], (st / kScanStages) & 1, kWaitTries)) {
+    uint64_t* bar = &bars[warp];
+    const uint8_t* tile = ring + warp * kBoxBytes;
+    for (int st = warp; st < nst; st += kScanStages) {
+        if (!ptx::mbar_wait_bounded(bar, (st / kScanStages) & 1, kWaitTries)) {
             ok = false;
-            if (tid == 0) record_error(P.status, kDevTimeout);
+            if (lane == 0) record_error(P.status, kDevTimeout);
+            break;
         }
-        float* ssc = stage_sc + (st & 1) * kScanRows;
-        if (ok) {
-            const uint8_t* tile = ring + buf * kBoxBytes;
-            const int row0 = warp * 16 + gid;
+        const int box0 = k0 + st * kScanRows;
+#pragma unroll 2
+        for (int rt = 0; rt < kScanRows / 16; ++rt) {
+            const int row0 = rt * 16 + gid;
             uint32_t ra[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = row0 + 8 * h;
                 uint4 u0, u1;
-                if (k0 + st * kScanRows + row == p) {
+                if (box0 + row == p) {
                     const uint4* src =
                         reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * kDI + 16 * tq);
                     u0 = src[0];
@@ -336,9 +343,9 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             }
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint32_t a[4] = {ra[0][2 * s], ra[1][2 * s], ra[0][2 * s + 1], ra[1][2 * s + 1]};
-                ptx::mma_bf16(acc, a, qb[2 * s], qb[2 * s + 1]);
+            for (int s4 = 0; s4 < 4; ++s4) {
+                const uint32_t a[4] = {ra[0][2 * s4], ra[1][2 * s4], ra[0][2 * s4 + 1], ra[1][2 * s4 + 1]};
+                ptx::mma_bf16(acc, a, qb[2 * s4], qb[2 * s4 + 1]);
             }
             float s0 = w_lo * fmaxf(acc[0], 0.0f) + w_hi * fmaxf(acc[1], 0.0f);
             float s1 = w_lo * fmaxf(acc[2], 0.0f) + w_hi * fmaxf(acc[3], 0.0f);
@@ -346,21 +353,22 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-            if (tq == 0) ssc[row0] = s0;
-            if (tq == 1) ssc[row0 + 8] = s1;
-        }
-        group_sync(kScanBar, kScanThreads);  // box consumed; this stage's scores in shared memory
-        if (tid == 0 && ok && st + kScanStages < nst) {
-            ptx::mbar_arrive_expect_tx(&bars[buf], kBoxBytes);
-            ptx::tma_load_2d(ring + buf * kBoxBytes, &tmap_kI, 0,
-                             b * P.N_max + k0 + (st + kScanStages) * kScanRows, &bars[buf]);
-        }
-        if (ok && tid < kScanRows) {
-            const int pos = k0 + st * kScanRows + tid;
-            if (pos < k1) {
-                const uint32_t kk = order_key(ssc[tid]);
+            // lane tq == 0 keeps key row0, tq == 1 key row0 + 8
+            const int pos = box0 + row0 + 8 * tq;
+            if (tq < 2 && pos < k1) {
+                const uint32_t kk = order_key(tq == 0 ? s0 : s1);
                 srow[pos] = kk;
                 atomicAdd(&lhist[kk >> 20], 1u);
+            }
+        }
+        if (st + kScanStages < nst) {
+            // the slot's reads are done: hand it back to the copy engine
+            __syncwarp();
+            if (lane == 0) {
+                ptx::fence_proxy_async_shared();
+                ptx::mbar_arrive_expect_tx(bar, kBoxBytes);
+                ptx::tma_load_2d(ring + warp * kBoxBytes, &tmap_kI, 0,
+                                 b * P.N_max + k0 + (st + kScanStages) * kScanRows, bar);
             }
         }
     }
@@ -371,10 +379,9 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (v) atomicAdd(&P.hist[(int64_t)b * 4096 + i], v);
     }
 
-    if (!ok && tid == 0) {
-        // give copies still in flight a bounded chance to land before exit
-        for (int i = 0; i < kScanStages; ++i)
-            for (uint32_t par = 0; par < 2; ++par) ptx::mbar_wait_bounded(&bars[i], par, 1u << 16);
+    if (!ok && lane == 0) {
+        // give this warp's copy still in flight a bounded chance to land before exit
+        for (uint32_t par = 0; par < 2; ++par) ptx::mbar_wait_bounded(bar, par, 1u << 16);
     }
 }
 
