@@ -79,55 +79,74 @@ struct AttOut {
     float o[8][4];
 };
 
+// Where the gathered K and V rows come from: the caches of one sequence
+// (row0 = b * N_max), except position p_special (if >= 0), which is read from
+// k_special / v_special; positions outside [0, p_max] are never dereferenced.
+struct AttSrc {
+    const __nv_bfloat16* k_cache;
+    const __nv_bfloat16* v_cache;
+    int64_t row0;
+    int p_max;
+    int p_special;
+    const __nv_bfloat16* k_special;
+    const __nv_bfloat16* v_special;
+};
+
+// The position this thread copies in stage st of the list pos[0..cnt) (the
+// stage's first entry pads a short last stage; those keys are masked).
+template <int HKV>
+__device__ __forceinline__ int attn_stage_pos(const int* pos, int cnt, int st) {
+    using A = AttGeo<HKV>;
+    if (st * A::keys >= cnt) return 0;
+    const int jj = st * A::keys + threadIdx.x / A::tpk;
+    return pos[jj < cnt ? jj : st * A::keys];
+}
+
+// Issues this thread's 16-byte asynchronous copies of stage st into ring slot
+// st % kAttStages and records the stage's positions (-1 past the list).
+template <int HKV>
+__device__ __forceinline__ void attn_issue_stage(uint8_t* ring, int* spos, int cnt, int st, int raw,
+                                                 const AttSrc& src) {
+    using A = AttGeo<HKV>;
+    using bf16 = __nv_bfloat16;
+    constexpr int GK = A::keys;
+    constexpr int kb_row = HKV * 128;
+    const int ck = threadIdx.x / A::tpk, sub = threadIdx.x % A::tpk;
+    uint8_t* dst = ring + (st % kAttStages) * A::stage_bytes;
+    if (sub == 0) spos[(st % kAttStages) * GK + ck] = (st * GK + ck < cnt) ? raw : -1;
+    const int ps = (raw < 0 || raw > src.p_max) ? 0 : raw;  // never dereference out of range
+    const bf16* ksrc = (ps == src.p_special) ? src.k_special : src.k_cache + (src.row0 + ps) * kb_row;
+    const bf16* vsrc = (ps == src.p_special) ? src.v_special : src.v_cache + (src.row0 + ps) * kb_row;
+#pragma unroll
+    for (int u = 0; u < A::cpt; ++u) {
+        const int i = sub + u * A::tpk;
+        const int which = i / A::rpc, off = i % A::rpc;
+        const bf16* from = which ? vsrc : ksrc;
+        ptx::cp_async_16(dst + which * GK * A::krow + ck * A::krow + off * 16,
+                         reinterpret_cast<const uint4*>(from) + off);
+    }
+}
+
 // q: the row's query fragments (attn_load_q), `group` <= 8 heads per KV
-// head.  pos[0..cnt): positions (shared or global memory).  Position
-// `p_special` (if >= 0) is read from k_special / v_special instead of the
-// caches.  Positions outside [0, p_max] are masked out and reported through
+// head.  pos[0..cnt): positions (shared or global memory), gathered from
+// `src`; positions outside [0, src.p_max] are masked out and reported through
 // `status`.  `ring` holds AttGeo<HKV>::ring_bytes bytes, `spos` (shared
 // memory) kAttStages * AttGeo<HKV>::keys ints; both are clobbered.  The
 // result is valid in the warps with part == 0 (warp % wph == 0).
 template <int HKV>
 __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spos, const int* pos,
-                                          int cnt, const __nv_bfloat16* k_cache,
-                                          const __nv_bfloat16* v_cache,
-                                          int64_t row0,  // b * N_max
-                                          int p_max, int p_special,
-                                          const __nv_bfloat16* k_special,
-                                          const __nv_bfloat16* v_special, float scale_log2,
+                                          int cnt, const AttSrc& src, float scale_log2,
                                           unsigned* status, AttOut& out) {
     using A = AttGeo<HKV>;
-    using bf16 = __nv_bfloat16;
     constexpr int GK = A::keys;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
     const int g_w = warp / A::wph, part = warp % A::wph;
     const int key0 = part * 16;  // this warp's keys within a stage
     const int nst = (cnt + GK - 1) / GK;
-    constexpr int kb_row = HKV * 128;
-
-    // copy role: thread copies chunks sub, sub + tpk, ... of key ck's K and V rows
-    const int ck = tid / A::tpk, sub = tid % A::tpk;
-    // position of key ck of stage st (a listed row pads the last stage; masked below)
-    auto load_pos = [&](int st) -> int {
-        if (st * GK >= cnt) return 0;
-        const int jj = st * GK + ck;
-        return pos[jj < cnt ? jj : st * GK];
-    };
-    auto issue_stage = [&](int st, int raw) {
-        uint8_t* dst = ring + (st % kAttStages) * A::stage_bytes;
-        if (sub == 0) spos[(st % kAttStages) * GK + ck] = (st * GK + ck < cnt) ? raw : -1;
-        const int ps = (raw < 0 || raw > p_max) ? 0 : raw;  // never dereference out of range
-        const bf16* ksrc = (ps == p_special) ? k_special : k_cache + (row0 + ps) * kb_row;
-        const bf16* vsrc = (ps == p_special) ? v_special : v_cache + (row0 + ps) * kb_row;
-#pragma unroll
-        for (int u = 0; u < A::cpt; ++u) {
-            const int i = sub + u * A::tpk;
-            const int which = i / A::rpc, off = i % A::rpc;
-            const bf16* src = which ? vsrc : ksrc;
-            ptx::cp_async_16(dst + which * GK * A::krow + ck * A::krow + off * 16,
-                             reinterpret_cast<const uint4*>(src) + off);
-        }
-    };
+    const int p_max = src.p_max;
+    auto load_pos = [&](int st) { return attn_stage_pos<HKV>(pos, cnt, st); };
+    auto issue_stage = [&](int st, int raw) { attn_issue_stage<HKV>(ring, spos, cnt, st, raw, src); };
 
     float* m = out.m;  // heads 2tq, 2tq + 1
     float* l = out.l;

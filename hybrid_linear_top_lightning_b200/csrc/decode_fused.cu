@@ -1,6 +1,6 @@
-// LISA decode step for B200 (sm_100a): three kernels chained by programmatic
-// dependent launch (each starts launching while its predecessor runs), every
-// SM busy, no inter-CTA waiting.
+// LISA decode step for B200 (sm_100a): four kernels chained by programmatic
+// dependent launch (each starts launching while its predecessor runs), no
+// inter-CTA waiting.
 //
 // Step semantics (LISA, arXiv 2607.19358v1: the generation step of Sec. 3.2 and
 // Eq. 1; Sec. 3.1 and Sec. 3.3 Eq. 3-4 for the linear branch): append the new
@@ -9,25 +9,24 @@
 //
 // K1 scan (grid B x S1, 8 scan warps + 4 linear-branch warps per CTA).
 //    Scan warps: CTA j of sequence b scores keys [j*KPC, (j+1)*KPC).  The k_I
-//    rows arrive by TMA (128-row boxes, 128-byte swizzle, eight in flight); a
-//    warp scores 16 keys at a time on the tensor cores (mma m16n8k16: keys x
-//    indexer heads, K = d_I), then ReLU, head weights and head sum.  Scores go
-//    to a workspace row; each slice also adds its histogram of the top 12 bits
-//    of the order-preserving score keys into the sequence's histogram.
+//    rows arrive by TMA (128-row boxes, 128-byte swizzle); scan warp w owns
+//    ring slot w and scores whole boxes on the tensor cores (mma m16n8k16:
+//    keys x indexer heads, K = d_I), then ReLU, head weights and head sum.
+//    The order-preserving keys of the scores go to a workspace row; each CTA
+//    adds its histogram of the keys' top 12 bits into the sequence's histogram.
 //    Linear-branch warps (concurrently): one slice (sequence, KV head, 32
 //    value columns) of S += phi(k)^T v and o_lin = phi(q) S (/ phi(q).z).
 //    CTA 0 of each sequence appends the new k, v, k_I to the caches.
-// K2 attend (grid B x S2, 256 threads).  Each CTA derives the exact top-M set
-//    by itself: the first 12-bit digit from the histogram, then one ordered
-//    pass over the score row (TMA-loaded into shared memory) collecting the
-//    keys of that digit, two 10-bit refinements over those candidates only,
-//    and a ranked walk (warp ballots and scans) that extracts this CTA's even
-//    share of the selected positions.  Ties keep the lowest positions.  The
-//    share's K and V rows (all KV heads of a position are one row) are
-//    gathered with 128-bit loads through registers into padded shared-memory
-//    rows and attended with an online softmax on the tensor cores.  Partial
-//    (max, sum, output) triples go to the workspace.
-// K3 combine (grid B x H_q, one thread per output dim): merges the partials,
+// K2 select (grid B, 1024 threads): the exact top-M of the key row (radix
+//    select: the 12-bit digit from the histogram, two 10-bit refinements over
+//    the keys of the threshold digit, ranks in position order; ties keep the
+//    lowest positions), written once as the sequence's index row.
+// K3 attend (grid B x S2, 256 threads): CTA j takes ranks [j*per, (j+1)*per)
+//    of the index row; their K and V rows (all KV heads of a position are one
+//    row) are gathered by cp.async into a shared-memory ring and attended with
+//    an online softmax on the tensor cores.  Partial (max, sum, output) triples
+//    go to the workspace.
+// K4 combine (grid B x H_q, one thread per output dim): merges the partials,
 //    gates with the linear branch, writes o; advances z (elu+1 mode) and clears
 //    the histogram for the next call.
 //
@@ -426,6 +425,16 @@ __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
     // over the keys that share the digits found so far.  Ties at the M-th key
     // keep the lowest positions.
     const uint32_t* srow = P.keys + (int64_t)b * P.ns;
+    SelectSmem sel;
+    sel.hist = reinterpret_cast<unsigned*>(sel_raw + SelSmem::hist);
+    sel.bc = reinterpret_cast<int*>(sel_raw + SelSmem::bc);
+    sel.cand = reinterpret_cast<uint2*>(sel_raw + SelSmem::cand);
+    if (n <= kSelRound) {
+        // every thread holds its 16 keys in registers, read from L2
+        row_topm<kSelNT, true>(srow, false, n, P.M, P.hist + (int64_t)b * 4096, sel, 0, P.M, out,
+                               nullptr, P.status);
+        return;
+    }
     const bool resident = n <= kSelKeyCap;
     if (resident && tid == 0) {
         const int bytes = ((n + 3) / 4) * 16;
@@ -434,10 +443,6 @@ __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
             ptx::bulk_load(reinterpret_cast<uint8_t*>(row_smem) + off, srow + off / 4,
                            min(16384, bytes - off), rowbar);
     }
-    SelectSmem sel;
-    sel.hist = reinterpret_cast<unsigned*>(sel_raw + SelSmem::hist);
-    sel.bc = reinterpret_cast<int*>(sel_raw + SelSmem::bc);
-    sel.cand = reinterpret_cast<uint2*>(sel_raw + SelSmem::cand);
     row_topm<kSelNT>(resident ? row_smem : srow, resident, n, P.M, P.hist + (int64_t)b * 4096, sel,
                      0, P.M, out, resident ? rowbar : nullptr, P.status);
 }
@@ -470,9 +475,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     // ---- gather + attention over this CTA's share of the selected positions
     constexpr int kb_row = HKV * kD;
     AttOut r;
-    attn_core<HKV>(q, att_raw + A::ring, spos, P.sel + (int64_t)b * P.M + lo, mine, P.k_cache,
-                   P.v_cache, (int64_t)b * P.N_max, p, p, P.k_new + (int64_t)b * kb_row,
-                   P.v_new + (int64_t)b * kb_row, P.scale_log2, P.status, r);
+    const AttSrc src{P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p, P.k_new + (int64_t)b * kb_row,
+                     P.v_new + (int64_t)b * kb_row};
+    attn_core<HKV>(q, att_raw + A::ring, spos, P.sel + (int64_t)b * P.M + lo, mine, src,
+                   P.scale_log2, P.status, r);
     // partial (m, l, O) of this CTA for every query head, from the first warp
     // of each KV head
     const int lane = tid & 31, warp = tid >> 5;

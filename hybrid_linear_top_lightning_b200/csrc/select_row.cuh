@@ -106,12 +106,14 @@ __device__ __forceinline__ uint64_t sel_lowest_bits(uint64_t m, int keep) {
 
 // row: the order-preserving keys (order_key) of n scores, resident in shared
 // memory (`resident`) or in global memory; the row buffer holds at least
-// round_up(n, 4) entries.  M < n.  first_hist:
+// round_up(n, 4) entries.  With REG (one round: n <= kSelRound), each thread
+// reads its chunk once into registers and every pass works from there.
+// M < n.  first_hist:
 // 4096-bin histogram of key >> 20 over the row, or null.  row_bar: if not
 // null, an mbarrier (phase 0) that completes when a TMA copy of the row into
 // shared memory has landed; it is waited on (bounded) before the row is read,
 // after the first digit when that comes from first_hist.
-template <int NT>
+template <int NT, bool REG = false>
 __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const unsigned* first_hist,
                          const SelectSmem& sm, int lo, int hi, int* out, uint64_t* row_bar,
                          unsigned* status) {
@@ -131,6 +133,31 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
         const uint4 v = resident ? *src : __ldg(src);
         k[0] = v.x; k[1] = v.y; k[2] = v.z; k[3] = v.w;
     };
+    // REG: the thread's chunk of round 0, read once (words in natural order)
+    uint32_t kr[REG ? kChunk : 1];
+    if (REG) {
+#pragma unroll
+        for (int j = 0; j < kQ; ++j) {
+            const int q = tid * kQ + j;
+            uint32_t k[4] = {0u, 0u, 0u, 0u};
+            if (4 * q < n) load4(q, k);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kr[(4 * j + e) % (REG ? kChunk : 1)] = k[e];
+        }
+    }
+    // word j of round r: its index q and its four keys
+    auto word = [&](int r, int j, uint32_t (&k)[4]) -> int {
+        if (REG) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) k[e] = kr[(4 * j + e) % (REG ? kChunk : 1)];
+            return tid * kQ + j;
+        }
+        const int q = chunk_q(r, j);
+        if (4 * q < n) load4(q, k);
+        return q;
+    };
+    // bit of word j's first key in the thread's chunk masks
+    auto word_bit = [&](int j) { return (REG ? j : ((j + tid) & (kQ - 1))) * 4; };
     auto wait_row = [&]() {
         if (!row_bar) return;
         bool ok = false;
@@ -167,12 +194,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
             for (int i = tid; i < 4096; i += NT) sm.hist[i] = 0u;
             __syncthreads();
             for (int r = 0; r < rounds; ++r)
-#pragma unroll 4
+#pragma unroll
                 for (int j = 0; j < kQ; ++j) {
-                    const int q = chunk_q(r, j);
-                    if (4 * q >= n) continue;
                     uint32_t k[4];
-                    load4(q, k);
+                    const int q = word(r, j, k);
+                    if (4 * q >= n) continue;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         if (4 * q + e < n) atomicAdd(&sm.hist[k[e] >> 20], 1u);
@@ -194,12 +220,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
     int ncand, above = 0, mine = 0, off;
     {
         for (int r = 0; r < rounds; ++r)
-#pragma unroll 4
+#pragma unroll
             for (int j = 0; j < kQ; ++j) {
-                const int q = chunk_q(r, j);
-                if (4 * q >= n) continue;
                 uint32_t k[4];
-                load4(q, k);
+                const int q = word(r, j, k);
+                if (4 * q >= n) continue;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const bool v = 4 * q + e < n;
@@ -211,12 +236,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
         if (ncand <= kCandTotal && mine > 0) {
             int w = off;
             for (int r = 0; r < rounds; ++r)
-#pragma unroll 4
+#pragma unroll
                 for (int j = 0; j < kQ; ++j) {
-                    const int q = chunk_q(r, j);
-                    if (4 * q >= n) continue;
                     uint32_t k[4];
-                    load4(q, k);
+                    const int q = word(r, j, k);
+                    if (4 * q >= n) continue;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         if ((4 * q + e < n) && (k[e] >> 20) == b1)
@@ -241,11 +265,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
             }
         } else {
             for (int r = 0; r < rounds; ++r)
+#pragma unroll
                 for (int j = 0; j < kQ; ++j) {
-                    const int q = chunk_q(r, j);
-                    if (4 * q >= n) continue;
                     uint32_t k[4];
-                    load4(q, k);
+                    const int q = word(r, j, k);
+                    if (4 * q >= n) continue;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         if (4 * q + e < n && (k[e] & mask) == prefix)
@@ -278,12 +302,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
     // `keep` = how many of its keys equal to tau are kept (its lowest ones)
     auto emit = [&](int r, int rank, int keep) {
         uint64_t gtm = 0, eqm = 0;
-#pragma unroll 4
+#pragma unroll
         for (int j = 0; j < kQ; ++j) {
-            const int q = chunk_q(r, j);
-            if (4 * q >= n) continue;
             uint32_t k[4];
-            load4(q, k);
+            const int q = word(r, j, k);
+            if (4 * q >= n) continue;
             const int nv = min(4, n - 4 * q);
             uint32_t g = 0, e4 = 0;
 #pragma unroll
@@ -291,7 +314,7 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
                 g |= (uint32_t)(e < nv && k[e] > tau) << e;
                 e4 |= (uint32_t)(e < nv && k[e] == tau) << e;
             }
-            const int bit = ((j + tid) & (kQ - 1)) * 4;
+            const int bit = word_bit(j);
             gtm |= (uint64_t)g << bit;
             eqm |= (uint64_t)e4 << bit;
         }
@@ -334,12 +357,11 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
 #pragma unroll 1
     for (int r = 0; r < rounds && rank_base < hi; ++r) {
         int gt_t = 0, eq_t = 0;
-#pragma unroll 4
+#pragma unroll
         for (int j = 0; j < kQ; ++j) {
-            const int q = chunk_q(r, j);
-            if (4 * q >= n) continue;
             uint32_t k[4];
-            load4(q, k);
+            const int q = word(r, j, k);
+            if (4 * q >= n) continue;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const bool v = 4 * q + e < n;

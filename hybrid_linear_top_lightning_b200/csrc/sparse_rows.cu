@@ -44,8 +44,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_sparse_rows(const SpParams P
     const int* pos = P.idx + (int64_t)row * P.M;  // read through L1 by the gather
     const AttQ q = attn_load_q<HKV>(P.q + (int64_t)row * P.H_q * 128, P.group);
     AttOut r;
-    attn_core<HKV>(q, sp_raw + L::ring, spos, pos, cnt, P.k, P.v, (int64_t)b * P.N_max, p, -1,
-                   nullptr, nullptr, P.scale_log2, P.status, r);
+    const AttSrc kv{P.k, P.v, (int64_t)b * P.N_max, p, -1, nullptr, nullptr};
+    attn_core<HKV>(q, sp_raw + L::ring, spos, pos, cnt, kv, P.scale_log2, P.status, r);
     // normalised output of each KV head's query heads (group rows of 128 dims,
     // contiguous in o), staged by the head's first warp in its own slot of the
     // ring and stored with 16-byte writes
