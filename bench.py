@@ -150,6 +150,26 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device=None, world: int = 1) -> float:
+    """The maximum of x over all ranks of the default process group (x itself
+    when there is only one rank): a multi-rank time is the slowest rank's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over all timed
+    steps, divided by the slowest rank's time."""
+    return world * units_per_rank * steps / (total_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def _setup_decode(wl, device):
     import torch
@@ -246,11 +266,7 @@ def run_gpu(args, wl, rank, world, device):
     times_ms = [s_.elapsed_time(e) for s_, e in zip(starts, ends)]
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
-    total_ms = sum(times_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(times_ms), device, world)
 
     # ---- end to end through the public API with host buffers
     pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
@@ -279,17 +295,13 @@ def run_gpu(args, wl, rank, world, device):
         e2e_step(i)
         e_en[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s_.elapsed_time(e) for s_, e in zip(e_st, e_en))
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(s_.elapsed_time(e) for s_, e in zip(e_st, e_en)), device, world)
 
     bytes_ = decode_bytes(wl)
     avg_s = total_ms / 1e3 / args.steps
     hbm_peak, _, peak_kind = _peaks()
     achieved = bytes_["total"] / avg_s / 1e9
-    value = world * B * args.steps / (total_ms / 1e3)
+    value = job_throughput(B, world, args.steps, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -311,7 +323,7 @@ def run_gpu(args, wl, rank, world, device):
                      "kernel": "decode step: one lisa_decode_step call = k_decode_scan + "
                                "k_decode_attend + k_decode_combine (PDL-chained)",
                      "launch_us": avg_s * 1e6},
-        "e2e": {"value": world * B * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": job_throughput(B, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),

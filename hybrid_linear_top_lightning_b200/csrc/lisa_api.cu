@@ -245,6 +245,8 @@ lisa_status lisa_gate_fuse(const lisa_dims* dims, const void* gate_logit_lin, co
     const Shape s = resolve(*dims);
     if ((int64_t)s.B * s.T == 0) return LISA_OK;
     if (!gate_logit_lin || !o_lin || !o_sparse || !o) return LISA_ERR_INVALID_ARG;
+    if (fast_gate_supported(s, o_lin, o_sparse, o))
+        return cuda_status(fast_gate(s, gate_logit_lin, o_lin, o_sparse, o, (cudaStream_t)stream));
     return cuda_status(generic_gate(s, gate_logit_lin, o_lin, false, o_sparse, false, o,
                                     (cudaStream_t)stream));
 }

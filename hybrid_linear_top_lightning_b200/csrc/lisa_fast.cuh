@@ -34,4 +34,10 @@ bool fast_linear_prefill_supported(const Shape& s, const void* q, const void* k,
 cudaError_t fast_linear_prefill(const Shape& s, const void* q, const void* k, const void* v,
                                 float* S, float* z, void* o, void* ws, cudaStream_t st);
 
+
+// gate_fast.cu: o = g o_lin + (1 - g) o_sparse for bf16 tensors, head dim 128
+bool fast_gate_supported(const Shape& s, const void* o_lin, const void* o_sp, const void* o);
+cudaError_t fast_gate(const Shape& s, const void* logit, const void* o_lin, const void* o_sp,
+                      void* o, cudaStream_t st);
+
 }  // namespace lisa
