@@ -70,17 +70,24 @@ def decode_bytes(wl) -> dict:
                 total=per_seq * wl.B)
 
 
+DECODE_KERNELS_PER_STEP = 4  # scan, select, attend, combine
+DECODE_SOURCES = ("decode_fused.cu", "attend_core.cuh", "select_row.cuh", "sm100_ptx.cuh",
+                  "tma_host.cuh", "lisa_internal.cuh")
+
+
 def _kernel_source_hash() -> str:
+    """Hash of the sources the decode-step kernels are compiled from: a
+    recorded DRAM traffic figure applies only to the kernels it was taken on."""
     h = hashlib.sha256()
-    for name in ("decode_fused.cu", "sm100_ptx.cuh", "lisa_internal.cuh"):
+    for name in DECODE_SOURCES:
         with open(os.path.join(ROOT, "hybrid_linear_top_lightning_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def _profiled_traffic(wl):
-    """DRAM bytes per launch of the fused decode kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+    """DRAM bytes of one decode step (its four kernels) from the committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", "decode_fused_traffic.json")
     try:
         with open(path) as f:
@@ -314,18 +321,19 @@ def run_gpu(args, wl, rank, world, device):
                          f"(caches, state, inputs) used in rotation, "
                          f"{args.rotate} x {bytes_['total'] / 1e6:.1f} MB touched per cycle",
                    "step": "decode step: append, linear update+readout, indexer scan, "
-                           "top-M, sparse attention, gate (3 kernels, PDL-chained)"},
+                           "top-M, sparse attention, gate (4 kernels, PDL-chained)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "frac_of_8TBs": achieved / 8000.0,
                      "traffic": _profiled_traffic(wl),
                      "algorithmic_bytes_per_launch": bytes_["total"],
                      "kernel": "decode step: one lisa_decode_step call = k_decode_scan + "
-                               "k_decode_attend + k_decode_combine (PDL-chained)",
+                               "k_decode_select + k_decode_attend + k_decode_combine "
+                               "(PDL-chained)",
                      "launch_us": avg_s * 1e6},
         "e2e": {"value": job_throughput(B, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": DECODE_KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
         "step_ms_min": min(times_ms), "step_ms_median": statistics.median(times_ms),
     }
