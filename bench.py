@@ -11,8 +11,11 @@ Timing: W untimed warm-up steps, then K steps, each timed with CUDA events on
 the launching stream.  Instead of flushing L2, the inputs are larger than L2:
 four copies of the whole decode state (caches, linear state, step inputs) at
 distinct addresses are used in rotation, so each step's ~55 MB of traffic was
-last touched three steps (~165 MB, more than the 126 MB L2) earlier.  A barrier and a device synchronise bracket the timed
-region; the reported time is the maximum over ranks.  Under torchrun each rank
+last touched three steps (~165 MB, more than the 126 MB L2) earlier.  Each timed
+step replays a CUDA graph captured from the lisa_decode_step call of its state
+copy (`--no-graphs`: the call itself); the end-to-end line calls the API
+directly.  A barrier and a device synchronise bracket the timed region; the
+reported time is the maximum over ranks.  Under torchrun each rank
 runs its own replica of the workload (weak scaling; the path has no exchange).
 
 `--impl reference` times the CPU oracle (plain fp64 C++) on the host cores on
@@ -252,6 +255,24 @@ def run_gpu(args, wl, rank, world, device):
     torch.cuda.synchronize()
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
+    if args.graphs:
+        # one CUDA graph per state copy, captured from the same call: a timed
+        # step is one graph launch, so the host's launch cost stays off the GPU
+        for c in copies:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                lisa.lisa_decode_step(D, c["a"], c["ws"])
+            c["graph"] = g
+        stream = torch.cuda.current_stream()
+
+        def step(i):  # noqa: F811
+            copies[i % len(copies)]["graph"].replay()
+
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        for c in copies:
+            assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -321,7 +342,9 @@ def run_gpu(args, wl, rank, world, device):
                          f"(caches, state, inputs) used in rotation, "
                          f"{args.rotate} x {bytes_['total'] / 1e6:.1f} MB touched per cycle",
                    "step": "decode step: append, linear update+readout, indexer scan, "
-                           "top-M, sparse attention, gate (4 kernels, PDL-chained)"},
+                           "top-M, sparse attention, gate (4 kernels, PDL-chained)",
+                   "launch": "CUDA graph replay of lisa_decode_step" if args.graphs
+                             else "lisa_decode_step from the host"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "frac_of_8TBs": achieved / 8000.0,
@@ -494,6 +517,9 @@ def main():
     ap.add_argument("--rotate", type=int, default=4,
                     help="copies of the decode state used in rotation (inputs larger than L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graphs", dest="graphs", action="store_false",
+                    help="launch every timed decode step from the host instead of replaying "
+                         "a captured CUDA graph")
     ap.add_argument("--prefill-steps", type=int, default=3,
                     help="timed calls per stage of the 7B prefill line (0: skip it)")
     ap.add_argument("--prefill-n", type=int, default=0,

@@ -12,23 +12,24 @@
 //    rows arrive by TMA (128-row boxes, 128-byte swizzle); scan warp w owns
 //    ring slot w and scores whole boxes on the tensor cores (mma m16n8k16:
 //    keys x indexer heads, K = d_I), then ReLU, head weights and head sum.
-//    The order-preserving keys of the scores go to a workspace row; each CTA
-//    adds its histogram of the keys' top 12 bits into the sequence's histogram.
+//    The order-preserving keys of the scores go to a workspace row, and each
+//    key's top 12 bits are counted into the sequence's histogram (global
+//    reductions issued as the keys are made).
 //    Linear-branch warps (concurrently): one slice (sequence, KV head, 32
 //    value columns) of S += phi(k)^T v and o_lin = phi(q) S (/ phi(q).z).
 //    CTA 0 of each sequence appends the new k, v, k_I to the caches.
 // K2 select (grid B, 1024 threads): the exact top-M of the key row (radix
 //    select: the 12-bit digit from the histogram, two 10-bit refinements over
 //    the keys of the threshold digit, ranks in position order; ties keep the
-//    lowest positions), written once as the sequence's index row.
+//    lowest positions), written once as the sequence's index row; clears the
+//    histogram for the next call.
 // K3 attend (grid B x S2, 256 threads): CTA j takes ranks [j*per, (j+1)*per)
 //    of the index row; their K and V rows (all KV heads of a position are one
 //    row) are gathered by cp.async into a shared-memory ring and attended with
 //    an online softmax on the tensor cores.  Partial (max, sum, output) triples
 //    go to the workspace.
 // K4 combine (grid B x H_q, one thread per output dim): merges the partials,
-//    gates with the linear branch, writes o; advances z (elu+1 mode) and clears
-//    the histogram for the next call.
+//    gates with the linear branch, writes o; advances z (elu+1 mode).
 //
 // The only waits are on TMA mbarriers, each bounded: a wait that gives up
 // records LISA_ERR_TIMEOUT in the status word and dependent work is skipped.
@@ -114,8 +115,7 @@ struct ScanSmem {
     static constexpr int vcol = fq + 16 * kD * 4;                    // float[32]
     static constexpr int zloc = vcol + kLaCols * 4;                  // float[128]
     static constexpr int den = zloc + kD * 4;                        // float[16]
-    static constexpr int lhist = den + 16 * 4;                       // u32[4096]
-    static constexpr int bars = lhist + 4096 * 4;                    // uint64[kScanStages]
+    static constexpr int bars = den + 16 * 4;                        // uint64[kScanStages]
     static constexpr int total = bars + kScanStages * 8 + 1024;      // + base alignment slack
 };
 
@@ -210,7 +210,6 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     float* vcol = reinterpret_cast<float*>(base + ScanSmem::vcol);
     float* zloc = reinterpret_cast<float*>(base + ScanSmem::zloc);
     float* den = reinterpret_cast<float*>(base + ScanSmem::den);
-    unsigned* lhist = reinterpret_cast<unsigned*>(base + ScanSmem::lhist);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + ScanSmem::bars);
 
     ptx::pdl_launch_dependents();
@@ -281,7 +280,6 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * kDI)[tid] = kin[tid];
         }
     }
-    for (int i = tid; i < 4096; i += kScanThreads) lhist[i] = 0u;
 
     // Indexer fragments.  mma m16n8k16 with A = 16 keys x 16 dims and B = 16 dims
     // x 8 heads; the thread (gid, tq) holds dims [16 tq, 16 tq + 16) of its rows
@@ -304,11 +302,11 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (2 * tq < P.H_I) w_lo = wb[2 * tq];
         if (2 * tq + 1 < P.H_I) w_hi = wb[2 * tq + 1];
     }
-    group_sync(kScanBar, kScanThreads);  // the local histogram is cleared
     // Warp w owns ring slot w: it scores boxes w, w + 8, ... by itself (8 row
-    // tiles of 16 keys each) and re-arms its slot, so no barrier joins the
-    // scan warps until the histogram is merged.
+    // tiles of 16 keys each) and re-arms its slot; no barrier joins the scan
+    // warps.
     uint32_t* srow = P.keys + (int64_t)b * P.ns;
+    unsigned* hist = P.hist + (int64_t)b * 4096;
     uint64_t* bar = &bars[warp];
     const uint8_t* tile = ring + warp * kBoxBytes;
     for (int st = warp; st < nst; st += kScanStages) {
@@ -357,7 +355,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             if (tq < 2 && pos < k1) {
                 const uint32_t kk = order_key(tq == 0 ? s0 : s1);
                 srow[pos] = kk;
-                atomicAdd(&lhist[kk >> 20], 1u);
+                atomicAdd(hist + (kk >> 20), 1u);  // a reduction: nothing waits for it
             }
         }
         if (st + kScanStages < nst) {
@@ -371,13 +369,6 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             }
         }
     }
-    // this slice's part of the sequence's 12-bit key histogram
-    group_sync(kScanBar, kScanThreads);
-    for (int i = tid; i < 4096; i += kScanThreads) {
-        const unsigned v = lhist[i];
-        if (v) atomicAdd(&P.hist[(int64_t)b * 4096 + i], v);
-    }
-
     if (!ok && lane == 0) {
         // give this warp's copy still in flight a bounded chance to land before exit
         for (uint32_t par = 0; par < 2; ++par) ptx::mbar_wait_bounded(bar, par, 1u << 16);
@@ -400,6 +391,13 @@ struct SelSmem {
     static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
 
+// Clears the key histogram of sequence b for the next call (once its reader,
+// the select kernel, no longer needs it).
+__device__ __forceinline__ void clear_hist(const Params& P, int b) {
+    uint4* hz = reinterpret_cast<uint4*>(P.hist + (int64_t)b * 4096);
+    for (int i = threadIdx.x; i < 4096 / 4; i += blockDim.x) hz[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
     extern __shared__ __align__(128) uint8_t sel_raw[];
     uint64_t* rowbar = reinterpret_cast<uint64_t*>(sel_raw + SelSmem::bar);
@@ -418,6 +416,7 @@ __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
     if (tid == 0 && P.count) P.count[b] = cnt;
     if (n <= P.M) {
         for (int i = tid; i < P.M; i += kSelNT) out[i] = i < n ? i : -1;
+        clear_hist(P, b);
         return;
     }
     // Radix select on the order-preserving score keys, most significant digit
@@ -433,6 +432,7 @@ __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
         // every thread holds its 16 keys in registers, read from L2
         row_topm<kSelNT, true>(srow, false, n, P.M, P.hist + (int64_t)b * 4096, sel, 0, P.M, out,
                                nullptr, P.status);
+        clear_hist(P, b);  // every read of it preceded row_topm's barriers
         return;
     }
     const bool resident = n <= kSelKeyCap;
@@ -445,7 +445,9 @@ __global__ void __launch_bounds__(kSelNT, 1) k_decode_select(const Params P) {
     }
     row_topm<kSelNT>(resident ? row_smem : srow, resident, n, P.M, P.hist + (int64_t)b * 4096, sel,
                      0, P.M, out, resident ? rowbar : nullptr, P.status);
+    clear_hist(P, b);
 }
+
 
 // ============================================================================ K3: attend
 template <int HKV>
@@ -505,52 +507,53 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
 // ============================================================================ K4: combine
 // One CTA per (sequence, query head), one thread per output dimension: merge
 // the attend CTAs' partial (max, sum, output) triples, mix with the linear
-// branch through the gate, write o.  Also advances the elu+1 normaliser z and
-// clears the sequence's key histogram for the next call.
+// branch through the gate, write o.  Also advances the elu+1 normaliser z.
 __global__ void __launch_bounds__(kD) k_decode_combine(const Params P) {
+    constexpr int kChunk = 32;  // partials loaded together
     const int b = blockIdx.x / P.H_q, h = blockIdx.x % P.H_q, c = threadIdx.x;
     ptx::pdl_wait_prior();  // the attend kernel's partials are complete
+    const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + h]);
+    const float o_lin = __ldcg(P.olin + ((int64_t)b * P.H_q + h) * kD + c);
     const int64_t jstride = (int64_t)P.H_q * (kD + 2);
     const float* rec0 = P.part + ((int64_t)b * P.S2 * P.H_q + h) * (kD + 2);
     float M = -INFINITY, Lsum = 0.0f, O = 0.0f;
 #pragma unroll 1
-    for (int j0 = 0; j0 < P.S2; j0 += 8) {
-        float mm[8], ll[8], oo[8];
+    for (int j0 = 0; j0 < P.S2; j0 += kChunk) {
+        float mm[kChunk], ll[kChunk], oo[kChunk];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kChunk; ++u) {
             mm[u] = -INFINITY;
             ll[u] = 0.0f;
             oo[u] = 0.0f;
             if (j0 + u < P.S2) {
                 const float* rec = rec0 + (j0 + u) * jstride;
-                mm[u] = __ldg(rec);
-                ll[u] = __ldg(rec + 1);
-                oo[u] = __ldg(rec + 2 + c);
+                mm[u] = __ldcg(rec);
+                ll[u] = __ldcg(rec + 1);
+                oo[u] = __ldcg(rec + 2 + c);
             }
         }
+        float cm = M;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            if (mm[u] == -INFINITY) continue;
-            const float nm = fmaxf(M, mm[u]);
-            const float a = exp2f(M - nm), w = exp2f(mm[u] - nm);
-            Lsum = fmaf(Lsum, a, ll[u] * w);
-            O = fmaf(O, a, oo[u] * w);
-            M = nm;
+        for (int u = 0; u < kChunk; ++u) cm = fmaxf(cm, mm[u]);
+        if (cm == -INFINITY) continue;
+        const float a = exp2f(M - cm);  // M = -inf gives 0
+        Lsum *= a;
+        O *= a;
+#pragma unroll
+        for (int u = 0; u < kChunk; ++u) {
+            const float wgt = exp2f(mm[u] - cm);  // an empty partial (-inf) weighs 0
+            Lsum = fmaf(ll[u], wgt, Lsum);
+            O = fmaf(oo[u], wgt, O);
         }
+        M = cm;
     }
     const float o_sp = Lsum > 0.0f ? O / Lsum : 0.0f;
-    const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + h]);
     const float gt = 1.0f / (1.0f + __expf(-x));
-    const float o_lin = __ldg(P.olin + ((int64_t)b * P.H_q + h) * kD + c);
     P.o[((int64_t)b * P.H_q + h) * kD + c] = __float2bfloat16_rn(gt * o_lin + (1.0f - gt) * o_sp);
     if (P.phi == LISA_PHI_ELU1_NORM && h < P.H_kv) {
         // z <- z + phi(k_L): every reader of the old z (the scan kernel) has finished
         const int64_t zi = ((int64_t)b * P.H_kv + h) * kD + c;
         P.z[zi] += feat(P.phi, __bfloat162float(P.k_L[zi]));
-    }
-    if (h == 0) {
-        uint4* hz = reinterpret_cast<uint4*>(P.hist + (int64_t)b * 4096);
-        for (int i = c; i < 4096 / 4; i += kD) hz[i] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
