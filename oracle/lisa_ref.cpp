@@ -336,4 +336,75 @@ int ref_forward(const RefDims* D, const float* q, const float* k_cache, const fl
     return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Sliding-window selection (Sec. 3.2, Stage 1: the sparse branch attends over
+// a fixed window of the last M positions before the Indexer replaces it):
+// query position p keeps [max(0, p-M+1), p], in ascending order, -1 padded.
+// idx: [B, R, M], count: [B, R].
+// ---------------------------------------------------------------------------
+void ref_window_indices(const RefDims* D, const int32_t* rows, int32_t R, int32_t* idx,
+                        int32_t* count) {
+    for (int b = 0; b < D->B; ++b) {
+        for (int r = 0; r < R; ++r) {
+            const int p = D->n_past + row_token(rows, r);
+            const int first = std::max(0, p - D->M + 1);
+            const int c = p - first + 1;
+            int32_t* out = idx + ((int64_t)b * R + r) * D->M;
+            for (int i = 0; i < D->M; ++i) out[i] = i < c ? first + i : -1;
+            count[(int64_t)b * R + r] = c;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Segment state transfer and correction at the end of reasoning segment t
+// (t >= 1), Sec. 3.3 Eq. 6-9, for every state matrix S[b, g] (d x d):
+//   grad_t    = S_end - S_start                  (Eq. 6; S_start = S_{t-1})
+//   mean_prev = grad_sum / (t - 1), or 0 at t = 1 (Eq. 7)
+//   grad_hat  = (1 - alpha) grad_t + alpha mean_prev        (Eq. 8)
+//   S_t       = S_start + grad_hat                          (Eq. 9)
+// In place: S (in: the state the segment's tokens reached; out: S_t),
+// S_start (out: S_t, the start of the next segment), grad_sum (out: the sum
+// of grad_1 .. grad_t).  All [B, H_kv, d, d].
+// ---------------------------------------------------------------------------
+void ref_state_transfer(const RefDims* D, double* S, double* S_start, double* grad_sum, int t,
+                        double alpha) {
+    const int64_t n = (int64_t)D->B * D->H_kv * D->d * D->d;
+    for (int64_t i = 0; i < n; ++i) {
+        const double grad_t = S[i] - S_start[i];
+        const double mean_prev = t > 1 ? grad_sum[i] / (t - 1) : 0.0;
+        const double grad_hat = (1.0 - alpha) * grad_t + alpha * mean_prev;
+        const double S_t = S_start[i] + grad_hat;
+        grad_sum[i] += grad_t;
+        S[i] = S_t;
+        S_start[i] = S_t;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per-channel gate (Sec. 3.3 Eq. 5): g = sigmoid(W_g h), one gate per output
+// channel (query head x dim), mixing the two branches as in Eq. 1:
+// o = g * o_LA + (1 - g) * o_SA_M.  h: [B, T, D_h]; W_g: [H_q*d, D_h];
+// o_lin, o_sp, o: [B, R, H_q, d].
+// ---------------------------------------------------------------------------
+void ref_gate_channel(const RefDims* D, int D_h, const float* h, const float* W_g,
+                      const int32_t* rows, int32_t R, const double* o_lin, const double* o_sp,
+                      double* o) {
+    const int N = D->H_q * D->d;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < D->B; ++b) {
+        for (int r = 0; r < R; ++r) {
+            const int t = row_token(rows, r);
+            const float* hv = h + ((int64_t)b * D->T + t) * D_h;
+            const int64_t base = ((int64_t)b * R + r) * N;
+            for (int c = 0; c < N; ++c) {
+                double x = 0.0;
+                for (int k = 0; k < D_h; ++k) x += (double)W_g[(int64_t)c * D_h + k] * hv[k];
+                const double g = 1.0 / (1.0 + std::exp(-x));
+                o[base + c] = g * o_lin[base + c] + (1.0 - g) * o_sp[base + c];
+            }
+        }
+    }
+}
+
 }  // extern "C"

@@ -167,3 +167,35 @@ def forward(D: Dims, q, k_cache, v_cache, q_I, k_I, w, w_tok_stride, q_L, k_L, v
                       ctypes.c_int64(w_tok_stride), _p(qL), _p(kL), _p(vL), _p(gl), _p(S), _p(z),
                       _p(r), ctypes.c_int32(R), _p(idx), _p(cnt), _p(o_sp), _p(o_lin), _p(o))
     return dict(idx=idx, count=cnt, o_sp=o_sp, o_lin=o_lin, o=o, S=S, z=z)
+
+
+def window_indices(D: Dims, rows=None):
+    """Sliding-window index rows (Stage 1): (idx [B,R,M] int32, count [B,R])."""
+    r, R = _rows(D, rows)
+    idx = np.empty((D.B, R, D.M), dtype=np.int32)
+    cnt = np.empty((D.B, R), dtype=np.int32)
+    lib().ref_window_indices(ctypes.byref(D.c()), _p(r), ctypes.c_int32(R), _p(idx), _p(cnt))
+    return idx, cnt
+
+
+def state_transfer(D: Dims, S_end, S_start, grad_sum, t: int, alpha: float):
+    """Segment state correction at the end of segment t (Eq. 6-9).
+    Returns (S_t, new S_start, new grad_sum), all fp64 copies."""
+    S = np.array(S_end, dtype=np.float64)
+    S0 = np.array(S_start, dtype=np.float64)
+    G = np.array(grad_sum, dtype=np.float64)
+    lib().ref_state_transfer(ctypes.byref(D.c()), _p(S), _p(S0), _p(G), ctypes.c_int(t),
+                             ctypes.c_double(alpha))
+    return S, S0, G
+
+
+def gate_channel(D: Dims, D_h: int, h, W_g, o_lin, o_sp, rows=None) -> np.ndarray:
+    """Per-channel gate (Eq. 5) mixing the two branches; o [B,R,H_q,d]."""
+    h, W_g = _f32(h), _f32(W_g)
+    r, R = _rows(D, rows)
+    o_lin = np.ascontiguousarray(o_lin, dtype=np.float64)
+    o_sp = np.ascontiguousarray(o_sp, dtype=np.float64)
+    out = np.empty_like(o_lin)
+    lib().ref_gate_channel(ctypes.byref(D.c()), ctypes.c_int(D_h), _p(h), _p(W_g), _p(r),
+                           ctypes.c_int32(R), _p(o_lin), _p(o_sp), _p(out))
+    return out
