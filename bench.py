@@ -244,7 +244,7 @@ def run_gpu(args, wl, rank, world, device):
         a = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"],
                              dv["w"], wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"],
                              kc, vc, kIc, S, None, o)
-        copies.append(dict(dv=dv, ws=ws, o=o, a=a))
+        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S))
 
     def step(i):
         c = copies[i % len(copies)]
@@ -325,6 +325,8 @@ def run_gpu(args, wl, rank, world, device):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(s_.elapsed_time(e) for s_, e in zip(e_st, e_en)), device, world)
 
+    extra = run_next_rows(args, wl, copies, D, stream) if args.next_rows else {}
+
     bytes_ = decode_bytes(wl)
     avg_s = total_ms / 1e3 / args.steps
     hbm_peak, _, peak_kind = _peaks()
@@ -360,7 +362,91 @@ def run_gpu(args, wl, rank, world, device):
         "clocks": clk.summary(),
         "step_ms_min": min(times_ms), "step_ms_median": statistics.median(times_ms),
     }
+    line.update(extra)
     return line
+
+
+# ----------------------------------------------------------------------------- next rows
+def window_bytes(wl) -> dict:
+    """Algorithmic HBM bytes of one sliding-window decode step: the last M K/V
+    rows (contiguous), the state read and written, the step's small tensors."""
+    M = min(wl.M, wl.n)
+    gather = M * wl.H_kv * wl.d * 2 * 2
+    state = wl.H_kv * wl.d * wl.d * 4 * 2
+    small = wl.H_q * wl.d * 2 * 3 + wl.H_kv * wl.d * 2 * 2 * 2 + wl.H_q * 2
+    per_seq = gather + state + small
+    return dict(per_seq=per_seq, total=per_seq * wl.B)
+
+
+def run_next_rows(args, wl, copies, D, stream):
+    """The Stage-1 sliding-window decode step and the segment state transfer,
+    on the same decode state: device-timed lines with their HBM rooflines."""
+    import torch
+
+    from hybrid_linear_top_lightning_b200 import lisa
+
+    hbm_peak, _, peak_kind = _peaks()
+    out = {}
+    # ---- sliding-window decode step (no indexer), graphs as for the main line
+    for c in copies:
+        lisa.lisa_decode_step_window(D, c["a"], c["ws"], stream)
+    torch.cuda.synchronize()
+    graphs = []
+    for c in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            lisa.lisa_decode_step_window(D, c["a"], c["ws"])
+        graphs.append(g)
+    cur = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i, (a_, b_) in enumerate(ev):
+        a_.record(cur)
+        graphs[i % len(graphs)].replay()
+        b_.record(cur)
+    torch.cuda.synchronize()
+    for c in copies:
+        assert lisa.lisa_check_status(c["ws"], cur) == lisa.LISA_OK
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / args.steps
+    wb = window_bytes(wl)
+    out["window"] = {
+        "what": "decode step with the Stage-1 sliding window (last M positions, no indexer): "
+                "lisa_decode_step_window, 3 kernels",
+        "value": wl.B / (ms / 1e3), "unit": "tok/s", "us_per_step": ms * 1e3,
+        "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": wb["total"],
+                     "achieved": wb["total"] / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": wb["total"] / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": None}}
+    # ---- segment state transfer over B x H_kv states of d x d fp32; 16 sets of
+    # (S, S_start, grad_sum) in rotation (201 MB, larger than L2)
+    shape = (wl.B, wl.H_kv, wl.d, wl.d)
+    states = [tuple(torch.randn(shape, device=stream.device) for _ in range(3)) for _ in range(16)]
+    for t in range(1, args.warmup + 1):
+        for S, S0, G in states:
+            lisa.lisa_state_transfer(D, S, S0, G, t, 0.25, stream)
+    torch.cuda.synchronize()
+    tms = []
+    for i in range(max(args.steps, 32)):
+        S, S0, G = states[i % len(states)]
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(cur)
+        lisa.lisa_state_transfer(D, S, S0, G, args.warmup + 1 + i // len(states), 0.25, stream)
+        b_.record(cur)
+        tms.append((a_, b_))
+    torch.cuda.synchronize()
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in tms) / len(tms)
+    st_bytes = 6 * wl.B * wl.H_kv * wl.d * wl.d * 4
+    out["state_transfer"] = {
+        "what": "segment state transfer and correction (Eq. 6-9) over B x H_kv states of d x d fp32",
+        "us_per_call": ms * 1e3, "l2": "16 state sets in rotation (201 MB, larger than L2)",
+        "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": st_bytes,
+                     "achieved": st_bytes / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": st_bytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": None}}
+    return out
 
 
 # ----------------------------------------------------------------------------- prefill
@@ -520,6 +606,8 @@ def main():
     ap.add_argument("--no-graphs", dest="graphs", action="store_false",
                     help="launch every timed decode step from the host instead of replaying "
                          "a captured CUDA graph")
+    ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
+                    help="skip the sliding-window step and state-transfer lines")
     ap.add_argument("--prefill-steps", type=int, default=3,
                     help="timed calls per stage of the 7B prefill line (0: skip it)")
     ap.add_argument("--prefill-n", type=int, default=0,

@@ -35,6 +35,7 @@
 // records LISA_ERR_TIMEOUT in the status word and dependent work is skipped.
 #include <cuda.h>
 #include <math.h>
+#include <string.h>
 
 #include <algorithm>
 
@@ -57,12 +58,14 @@ constexpr int kScanRows = 128;        // keys per TMA box (16 per warp)
 constexpr int kScanStages = 8;        // boxes in flight per CTA
 constexpr int kBoxBytes = kScanRows * kDI * 2;
 constexpr int kLaCols = 32;           // linear-state columns per slice
+constexpr int kMaxPer = 2048;         // positions per attend CTA in the window step
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
     int B, n, ns, N_max, H_q, H_kv, group, H_I, M, phi;
     int S1, KPC;        // scan CTAs per sequence, keys per scan CTA
     int S2, per;        // attend CTAs per sequence, selected positions per attend CTA
+    int window;         // 1: the sparse branch attends over the last M positions (no indexer)
     int la_slices;      // B * H_kv * (kD / kLaCols)
     int rowbytes;       // bytes of one cached K (or V) row: H_kv * kD * 2
     float scale_log2;   // sm_scale * log2(e)
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     const int n = P.n, p = n - 1;
     const int k0 = j * P.KPC;
     const int k1 = min(n, k0 + P.KPC);
-    const int nk = max(0, k1 - k0);
+    const int nk = P.window ? 0 : max(0, k1 - k0);  // the window step scans nothing
     const int nst = (nk + kScanRows - 1) / kScanRows;
     bool ok = true;
 
@@ -275,11 +278,13 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             kd[i] = kn[i];
             vd[i] = vn[i];
         }
-        if (tid < kDI / 8) {
+        if (!P.window && tid < kDI / 8) {
             const uint4* kin = reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * kDI);
             reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * kDI)[tid] = kin[tid];
         }
     }
+
+    if (P.window) return;  // no indexer in the sliding-window step
 
     // Indexer fragments.  mma m16n8k16 with A = 16 keys x 16 dims and B = 16 dims
     // x 8 heads; the thread (gid, tq) holds dims [16 tq, 16 tq + 16) of its rows
@@ -454,7 +459,8 @@ template <int HKV>
 struct Att : AttGeo<HKV> {
     using G = AttGeo<HKV>;
     static constexpr int spos = 0;                                     // int[stages][keys]
-    static constexpr int ring = (kAttStages * G::keys * 4 + 127) / 128 * 128;
+    static constexpr int wpos = (kAttStages * G::keys * 4 + 127) / 128 * 128;  // int[kMaxPer] (window step)
+    static constexpr int ring = wpos + kMaxPer * 4;
     static constexpr int total = ring + G::ring_bytes;
     static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
@@ -473,13 +479,29 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_decode_attend(const Params P
     const int cnt = min(P.M, n);
     const int lo = j * P.per, hi = min(cnt, lo + P.per);
     const int mine = max(0, hi - lo);
+    const int* pos = P.sel + (int64_t)b * P.M + lo;
+    if (P.window) {
+        // the last cnt positions; this CTA's share is [n - cnt + lo, n - cnt + hi)
+        int* wpos = reinterpret_cast<int*>(att_raw + A::wpos);
+        const int first = n - cnt + lo;
+        for (int i = tid; i < mine; i += kAttThreads) {
+            wpos[i] = first + i;
+            if (P.idx) P.idx[(int64_t)b * P.M + lo + i] = first + i;
+        }
+        if (j == 0) {
+            if (P.idx)
+                for (int i = cnt + tid; i < P.M; i += kAttThreads) P.idx[(int64_t)b * P.M + i] = -1;
+            if (P.count && tid == 0) P.count[b] = cnt;
+        }
+        pos = wpos;  // attn_core's first barrier publishes the list
+    }
 
     // ---- gather + attention over this CTA's share of the selected positions
     constexpr int kb_row = HKV * kD;
     AttOut r;
     const AttSrc src{P.k_cache, P.v_cache, (int64_t)b * P.N_max, p, p, P.k_new + (int64_t)b * kb_row,
                      P.v_new + (int64_t)b * kb_row};
-    attn_core<HKV>(q, att_raw + A::ring, spos, P.sel + (int64_t)b * P.M + lo, mine, src,
+    attn_core<HKV>(q, att_raw + A::ring, spos, pos, mine, src,
                    P.scale_log2, P.status, r);
     // partial (m, l, O) of this CTA for every query head, from the first warp
     // of each KV head
@@ -610,25 +632,29 @@ size_t fast_decode_ws_bytes(const Shape& s) {
     return make_plan(s).end;
 }
 
-bool fast_decode_supported(const Shape& s, const lisa_decode_args& a) {
-    if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD || s.d_I != kDI || s.H_Ik != 1) return false;
-    if (s.H_I > 8 || s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
+bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool window) {
+    if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD) return false;
+    if (!window && (s.d_I != kDI || s.H_Ik != 1 || s.H_I > 8)) return false;
+    if (s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
     if (s.L < 1 || s.M < 1 || s.B < 1) return false;
-    const void* ptrs[] = {a.q, a.k_new, a.v_new, a.q_I, a.k_I_new, a.q_L, a.k_L, a.v_L,
-                          a.k_cache, a.v_cache, a.k_I_cache, a.S, a.o};
+    if (window && make_plan(s).per > kMaxPer) return false;
+    const void* ptrs[] = {a.q, a.k_new, a.v_new, a.q_L, a.k_L, a.v_L, a.k_cache, a.v_cache, a.S, a.o};
     for (const void* p : ptrs)
         if (!aligned16(p)) return false;
+    if (!window && (!aligned16(a.q_I) || !aligned16(a.k_I_new) || !aligned16(a.k_I_cache)))
+        return false;
     if (s.phi == LISA_PHI_ELU1_NORM && !aligned16(a.z)) return false;
-    if (!tma_encode_fn()) return false;
+    if (!window && !tma_encode_fn()) return false;
     return true;
 }
 
-cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st) {
+cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
+                             bool window) {
     const Plan pl = make_plan(s);
     Params P;
     P.B = s.B; P.n = s.L; P.ns = pl.ns; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv;
     P.group = s.group; P.H_I = s.H_I; P.M = s.M; P.phi = s.phi;
-    P.S1 = pl.S1; P.KPC = pl.KPC; P.S2 = pl.S2; P.per = pl.per;
+    P.S1 = pl.S1; P.KPC = pl.KPC; P.S2 = pl.S2; P.per = pl.per; P.window = window ? 1 : 0;
     P.la_slices = s.B * s.H_kv * (kD / kLaCols);
     P.rowbytes = s.H_kv * kD * 2;
     P.scale_log2 = s.sm_scale * 1.4426950408889634f;
@@ -647,7 +673,8 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     P.sel = a.idx ? a.idx : (int32_t*)(w8 + pl.sel);
 
     CUtensorMap tmap;
-    if (!make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max, kScanRows))
+    memset(&tmap, 0, sizeof(tmap));  // unused by the window step (it scans no keys)
+    if (!window && !make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max, kScanRows))
         return cudaErrorInvalidValue;
 
     static bool attrs_set[64] = {};
@@ -684,11 +711,13 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(s.B);
-    cfg.blockDim = dim3(kSelNT);
-    cfg.dynamicSmemBytes = SelSmem::total;
-    e = cudaLaunchKernelEx(&cfg, k_decode_select, P);
-    if (e != cudaSuccess) return e;
+    if (!window) {
+        cfg.gridDim = dim3(s.B);
+        cfg.blockDim = dim3(kSelNT);
+        cfg.dynamicSmemBytes = SelSmem::total;
+        e = cudaLaunchKernelEx(&cfg, k_decode_select, P);
+        if (e != cudaSuccess) return e;
+    }
     cfg.gridDim = dim3(s.B * pl.S2);
     cfg.blockDim = dim3(kAttThreads);
     switch (s.H_kv) {

@@ -325,7 +325,27 @@ __global__ void k_append(int B, int n_past, int N_max, int width_kv, int width_k
         kIc[dst_kI + i] = kI_new[(int64_t)b * width_kI + i];
 }
 
+// Sliding-window rows (Sec. 3.2, Stage 1): token t at position p = n_past + t
+// keeps [max(0, p-M+1), p] in ascending order, -1 padded.
+__global__ void k_window_indices(int64_t rows, int T, int n_past, int M, int32_t* __restrict__ idx,
+                                 int32_t* __restrict__ count) {
+    const int64_t row = blockIdx.x;
+    if (row >= rows) return;
+    const int p = n_past + (int)(row % T);
+    const int first = max(0, p - M + 1);
+    const int c = p - first + 1;
+    for (int i = threadIdx.x; i < M; i += blockDim.x) idx[row * M + i] = i < c ? first + i : -1;
+    if (threadIdx.x == 0) count[row] = c;
+}
+
 }  // namespace
+
+cudaError_t generic_window_indices(const Shape& s, int32_t* idx, int32_t* count, cudaStream_t st) {
+    const int64_t rows = (int64_t)s.B * s.T;
+    if (rows == 0) return cudaSuccess;
+    k_window_indices<<<(unsigned)rows, 128, 0, st>>>(rows, s.T, s.n_past, s.M, idx, count);
+    return cudaGetLastError();
+}
 
 // ------------------------------------------------------------------ launchers
 cudaError_t generic_index_scores(const Shape& s, const void* q_I, const void* k_I, const float* w,
@@ -428,7 +448,7 @@ cudaError_t generic_append(const Shape& s, const void* k_new, const void* v_new,
                            const void* k_I_new, void* k_cache, void* v_cache, void* k_I_cache,
                            cudaStream_t st) {
     if (s.B == 0) return cudaSuccess;
-    const int wkv = s.H_kv * s.d, wkI = s.H_Ik * s.d_I;
+    const int wkv = s.H_kv * s.d, wkI = (k_I_new && k_I_cache) ? s.H_Ik * s.d_I : 0;
     if (s.dtype == LISA_BF16) {
         using T = __nv_bfloat16;
         k_append<T><<<s.B, 256, 0, st>>>(s.B, s.n_past, s.N_max, wkv, wkI, (const T*)k_new,

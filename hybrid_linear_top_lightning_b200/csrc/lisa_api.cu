@@ -313,6 +313,52 @@ lisa_status lisa_prefill(const lisa_dims* dims, const lisa_prefill_args* a, void
     return lisa_gate_fuse(dims, a->gate_logit_lin, o_lin, o_sp, a->o, stream);
 }
 
+lisa_status lisa_window_indices(const lisa_dims* dims, int32_t* idx, int32_t* count, void* stream) {
+    LISA_TRY(check_dims(dims));
+    const Shape s = resolve(*dims);
+    if ((int64_t)s.B * s.T == 0) return LISA_OK;
+    if (!idx || !count) return LISA_ERR_INVALID_ARG;
+    return cuda_status(generic_window_indices(s, idx, count, (cudaStream_t)stream));
+}
+
+lisa_status lisa_decode_step_window(const lisa_dims* dims, const lisa_decode_args* a, void* ws,
+                                    size_t ws_bytes, void* stream) {
+    LISA_TRY(check_dims(dims));
+    if (dims->T != 1 || !a) return LISA_ERR_INVALID_ARG;
+    const Shape s = resolve(*dims);
+    if (s.B == 0) return LISA_OK;
+    if (!a->q || !a->k_new || !a->v_new || !a->q_L || !a->k_L || !a->v_L || !a->gate_logit_lin ||
+        !a->k_cache || !a->v_cache || !a->S || !a->o)
+        return LISA_ERR_INVALID_ARG;
+    if (s.phi == LISA_PHI_ELU1_NORM && !a->z) return LISA_ERR_INVALID_ARG;
+    LISA_TRY(check_ws(ws, ws_bytes, workspace_bytes(s, LISA_OP_DECODE_STEP)));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (fast_decode_supported(s, *a, true)) return cuda_status(fast_decode_step(s, *a, ws, st, true));
+
+    const DecodeWs lay = decode_ws(s);
+    char* base = (char*)ws;
+    int32_t* idx = a->idx ? a->idx : (int32_t*)(base + lay.idx);
+    int32_t* count = a->count ? a->count : (int32_t*)(base + lay.count);
+    float* o_sp = (float*)(base + lay.o_sp);
+    float* o_lin = (float*)(base + lay.o_lin);
+    LISA_CUDA(generic_append(s, a->k_new, a->v_new, nullptr, a->k_cache, a->v_cache, nullptr, st));
+    LISA_CUDA(generic_linear(s, a->q_L, a->k_L, a->v_L, a->S, a->z, o_lin, true, st));
+    LISA_CUDA(generic_window_indices(s, idx, count, st));
+    LISA_CUDA(generic_attention(s, a->q, a->k_cache, a->v_cache, idx, count, o_sp, true,
+                                (unsigned*)ws, st));
+    return cuda_status(generic_gate(s, a->gate_logit_lin, o_lin, true, o_sp, true, a->o, st));
+}
+
+lisa_status lisa_state_transfer(const lisa_dims* dims, float* S, float* S_start, float* grad_sum,
+                                int32_t t, float alpha, void* stream) {
+    LISA_TRY(check_dims(dims));
+    if (t < 1 || !(alpha == alpha)) return LISA_ERR_INVALID_ARG;
+    const Shape s = resolve(*dims);
+    if ((int64_t)s.B * s.H_kv == 0) return LISA_OK;
+    if (!S || !S_start || !grad_sum) return LISA_ERR_INVALID_ARG;
+    return cuda_status(state_transfer(s, S, S_start, grad_sum, t, alpha, (cudaStream_t)stream));
+}
+
 lisa_status lisa_check_status(void* ws, void* stream) {
     if (!ws) return LISA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;

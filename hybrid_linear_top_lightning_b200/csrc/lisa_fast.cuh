@@ -9,8 +9,10 @@ namespace lisa {
 
 // Fused decode step (decode_fused.cu).
 size_t fast_decode_ws_bytes(const Shape& s);
-bool fast_decode_supported(const Shape& s, const lisa_decode_args& a);
-cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st);
+// window: the sparse branch attends over the last M positions (no indexer)
+bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool window = false);
+cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
+                             bool window = false);
 
 // Top-M over many query rows (prefill).
 size_t fast_topm_ws_bytes(const Shape& s);
@@ -39,5 +41,10 @@ cudaError_t fast_linear_prefill(const Shape& s, const void* q, const void* k, co
 bool fast_gate_supported(const Shape& s, const void* o_lin, const void* o_sp, const void* o);
 cudaError_t fast_gate(const Shape& s, const void* logit, const void* o_lin, const void* o_sp,
                       void* o, cudaStream_t st);
+
+
+// state_transfer.cu: segment state correction (Sec. 3.3 Eq. 6-9), any shape
+cudaError_t state_transfer(const Shape& s, float* S, float* S_start, float* grad_sum, int t,
+                           float alpha, cudaStream_t st);
 
 }  // namespace lisa

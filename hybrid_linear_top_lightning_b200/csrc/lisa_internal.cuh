@@ -60,6 +60,8 @@ cudaError_t generic_linear(const Shape& s, const void* q_L, const void* k_L, con
 // o = sigmoid(x) * o_lin + (1 - sigmoid(x)) * o_sp; branch inputs in act dtype or float32.
 cudaError_t generic_gate(const Shape& s, const void* logit, const void* o_lin, bool lin_f32,
                          const void* o_sp, bool sp_f32, void* o, cudaStream_t st);
+cudaError_t generic_window_indices(const Shape& s, int32_t* idx, int32_t* count, cudaStream_t st);
+// k_I_new / k_I_cache may be null: only k and v are appended
 cudaError_t generic_append(const Shape& s, const void* k_new, const void* v_new,
                            const void* k_I_new, void* k_cache, void* v_cache, void* k_I_cache,
                            cudaStream_t st);

@@ -41,7 +41,8 @@ EXPORTS = (
     "lisa_index_scores", "lisa_topm", "lisa_sparse_attn", "lisa_linear_prefill",
     "lisa_linear_decode", "lisa_gate_fuse", "lisa_decode_step", "lisa_dense_attn",
     "lisa_workspace_size", "lisa_check_status", "lisa_status_string", "lisa_version",
-    "lisa_topm_noalloc", "lisa_prefill",
+    "lisa_topm_noalloc", "lisa_prefill", "lisa_window_indices", "lisa_decode_step_window",
+    "lisa_state_transfer",
 )
 
 
@@ -107,6 +108,9 @@ def load() -> ctypes.CDLL:
         "lisa_check_status": [vp, vp],
         "lisa_topm_noalloc": [dp, vp, vp, vp, i64, vp, vp, vp],
         "lisa_prefill": [dp, ctypes.POINTER(lisa_prefill_args), vp, sz, vp],
+        "lisa_window_indices": [dp, vp, vp, vp],
+        "lisa_decode_step_window": [dp, ctypes.POINTER(lisa_decode_args), vp, sz, vp],
+        "lisa_state_transfer": [dp, vp, vp, vp, ctypes.c_int32, ctypes.c_float, vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -251,6 +255,21 @@ def prefill_args(q, k_cache, v_cache, q_I, k_I_cache, w, w_tok_stride, q_L, k_L,
 def lisa_prefill(dims, args: lisa_prefill_args, ws, stream=None):
     _check(load().lisa_prefill(ctypes.byref(dims), ctypes.byref(args), _ptr(ws), ws.numel(),
                                _stream(stream)), "lisa_prefill")
+
+
+def lisa_window_indices(dims, idx, count, stream=None):
+    _check(load().lisa_window_indices(ctypes.byref(dims), _ptr(idx), _ptr(count), _stream(stream)),
+           "lisa_window_indices")
+
+
+def lisa_decode_step_window(dims, args: lisa_decode_args, ws, stream=None):
+    _check(load().lisa_decode_step_window(ctypes.byref(dims), ctypes.byref(args), _ptr(ws),
+                                          ws.numel(), _stream(stream)), "lisa_decode_step_window")
+
+
+def lisa_state_transfer(dims, S, S_start, grad_sum, t: int, alpha: float, stream=None):
+    _check(load().lisa_state_transfer(ctypes.byref(dims), _ptr(S), _ptr(S_start), _ptr(grad_sum),
+                                      int(t), float(alpha), _stream(stream)), "lisa_state_transfer")
 
 
 def lisa_decode_step(dims, args: lisa_decode_args, ws, stream=None):

@@ -217,6 +217,44 @@ typedef struct lisa_prefill_args {
 LISA_API lisa_status lisa_prefill(const lisa_dims* dims, const lisa_prefill_args* args, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Beyond the main path: the Stage-1 sparse branch and the segment state update.
+ * ------------------------------------------------------------------------- */
+
+/* Sliding-window index rows (LISA Sec. 3.2, Stage 1, the branch the Indexer
+ * later replaces): token t at position p = n_past + t keeps the positions
+ * [max(0, p-M+1), p] in ascending order.  Same outputs and layout as
+ * lisa_topm (idx [B,T,M] int32, -1 padded; count [B,T] = min(M, p+1)); feed
+ * them to lisa_sparse_attn.  Uses B, T, n_past and M of dims. */
+LISA_API lisa_status lisa_window_indices(const lisa_dims* dims, int32_t* idx, int32_t* count,
+                                         void* stream);
+
+/* One decode step of the module with the Stage-1 sparse branch: as
+ * lisa_decode_step, but the sparse attention runs over the last min(M, n)
+ * positions instead of the Indexer's top-M (LISA Sec. 3.2 Eq. 1 with o_SA_M the
+ * sliding-window output).  q_I, k_I_new, k_I_cache and w are not used and may
+ * be NULL; the k_I cache is not appended.  idx/count, when given, receive the
+ * window.  Workspace: lisa_workspace_size(.., LISA_OP_DECODE_STEP). */
+LISA_API lisa_status lisa_decode_step_window(const lisa_dims* dims, const lisa_decode_args* args,
+                                             void* ws, size_t ws_bytes, void* stream);
+
+/* Segment state transfer and correction at the end of reasoning segment t
+ * (t >= 1; LISA Sec. 3.3, "Segment State Update", Eq. 6-9), for every state
+ * matrix S[b, g]:
+ *   grad_t   = S - S_start                           (Eq. 6, S_start = S_{t-1})
+ *   mean     = grad_sum / (t - 1), zero when t = 1   (Eq. 7)
+ *   grad_hat = (1 - alpha) grad_t + alpha mean       (Eq. 8)
+ *   S_t      = S_start + grad_hat                    (Eq. 9)
+ * In place, all fp32 [B, H_kv, d, d] device arrays: S (in: the state the
+ * segment's tokens reached; out: S_t), S_start (in: S_{t-1}; out: S_t, the
+ * start of the next segment), grad_sum (in: grad_1 + ... + grad_{t-1}, zeros
+ * before the first segment; out: the sum through grad_t).  alpha is the
+ * paper's correction coefficient (unstated there; a caller's parameter).
+ * Applies to S only: the elu+1 normaliser z is left as the tokens made it.
+ * Errors: LISA_ERR_INVALID_ARG for t < 1, a NaN alpha or a null pointer. */
+LISA_API lisa_status lisa_state_transfer(const lisa_dims* dims, float* S, float* S_start,
+                                         float* grad_sum, int32_t t, float alpha, void* stream);
+
 /* Dense causal softmax attention over every cached position s <= p (Sec. 3.1,
  * the standard attention LISA replaces); the O(n) reference line. */
 LISA_API lisa_status lisa_dense_attn(const lisa_dims* dims, const void* q, const void* k_cache,

@@ -401,7 +401,7 @@ void ref_gate_channel(const RefDims* D, int D_h, const float* h, const float* W_
                 double x = 0.0;
                 for (int k = 0; k < D_h; ++k) x += (double)W_g[(int64_t)c * D_h + k] * hv[k];
                 const double g = 1.0 / (1.0 + std::exp(-x));
-                o[base + c] = g * o_lin[base + c] + (1.0 - g) * o_sp[base + c];
+                o[base + c] = (1.0 - g) * o_sp[base + c] + g * o_lin[base + c];
             }
         }
     }
