@@ -244,7 +244,7 @@ def run_gpu(args, wl, rank, world, device):
         a = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"],
                              dv["w"], wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"],
                              kc, vc, kIc, S, None, o)
-        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S))
+        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S, kc=kc, vc=vc))
 
     def step(i):
         c = copies[i % len(copies)]
@@ -420,6 +420,58 @@ def run_next_rows(args, wl, copies, D, stream):
                      "achieved": wb["total"] / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": wb["total"] / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
                      "traffic": None}}
+    # ---- the paper's indexer form: a key per indexer head (H_Ik = H_I = 8), w = 1
+    from hybrid_linear_top_lightning_b200 import inputs
+
+    wl8 = wl.with_(H_Ik=wl.H_I)
+    gen8 = inputs.Generator(wl8)
+    n, p, B = wl.n, wl.n - 1, wl.B
+    kI8 = torch.empty(B, n, wl.H_I, wl.d_I, dtype=torch.bfloat16, device=stream.device)
+    for b in range(B):
+        kI8[b] = torch.from_numpy(gen8.k_I(b, 0, n)).to(torch.bfloat16)
+    D8 = lisa.make_dims(B, 1, p, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_I, wl.d_I, wl.M)
+    w1 = torch.ones(B, 1, wl.H_I, device=stream.device)
+    pf = []
+    for i, c in enumerate(copies):
+        kc8 = kI8 if i == 0 else kI8.clone()
+        kI_new = kc8[:, p:].clone()
+        dv = c["dv"]
+        a8 = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], kI_new, w1, wl.H_I,
+                              dv["q"], dv["k_new"], dv["v_new"], dv["gate"], c["kc"], c["vc"], kc8,
+                              c["S"], None, c["o"])
+        pf.append(dict(a=a8, ws=lisa.workspace(D8, lisa.LISA_OP_DECODE_STEP, stream.device)))
+    for c in pf:
+        lisa.lisa_decode_step(D8, c["a"], c["ws"], stream)
+    torch.cuda.synchronize()
+    for c in pf:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            lisa.lisa_decode_step(D8, c["a"], c["ws"])
+        c["graph"] = g
+    for i in range(args.warmup):
+        pf[i % len(pf)]["graph"].replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i, (a_, b_) in enumerate(ev):
+        a_.record(cur)
+        pf[i % len(pf)]["graph"].replay()
+        b_.record(cur)
+    torch.cuda.synchronize()
+    for c in pf:
+        assert lisa.lisa_check_status(c["ws"], cur) == lisa.LISA_OK
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / args.steps
+    pb = decode_bytes(wl8)
+    out["paper_form"] = {
+        "what": "decode step with the paper's indexer form: a key per indexer head "
+                "(H_Ik = H_I = 8, 1 KB of k_I per token), unweighted head sum",
+        "value": B / (ms / 1e3), "unit": "tok/s", "us_per_step": ms * 1e3,
+        "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": pb["total"],
+                     "achieved": pb["total"] / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": pb["total"] / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": None}}
+    del pf, kI8
+
     # ---- segment state transfer over B x H_kv states of d x d fp32; 16 sets of
     # (S, S_start, grad_sum) in rotation (201 MB, larger than L2)
     shape = (wl.B, wl.H_kv, wl.d, wl.d)
@@ -428,20 +480,27 @@ def run_next_rows(args, wl, copies, D, stream):
         for S, S0, G in states:
             lisa.lisa_state_transfer(D, S, S0, G, t, 0.25, stream)
     torch.cuda.synchronize()
-    tms = []
-    for i in range(max(args.steps, 32)):
-        S, S0, G = states[i % len(states)]
-        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_.record(cur)
-        lisa.lisa_state_transfer(D, S, S0, G, args.warmup + 1 + i // len(states), 0.25, stream)
-        b_.record(cur)
-        tms.append((a_, b_))
+    # one graph of 16 calls (a call is a few microseconds: shorter than a host launch)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for S, S0, G in states:
+            lisa.lisa_state_transfer(D, S, S0, G, args.warmup + 1, 0.25)
+    g.replay()
     torch.cuda.synchronize()
-    ms = sum(a_.elapsed_time(b_) for a_, b_ in tms) / len(tms)
+    reps = max(4, args.steps // 8)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a_, b_ in ev:
+        a_.record(cur)
+        g.replay()
+        b_.record(cur)
+    torch.cuda.synchronize()
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in ev) / (reps * len(states))
     st_bytes = 6 * wl.B * wl.H_kv * wl.d * wl.d * 4
     out["state_transfer"] = {
         "what": "segment state transfer and correction (Eq. 6-9) over B x H_kv states of d x d fp32",
-        "us_per_call": ms * 1e3, "l2": "16 state sets in rotation (201 MB, larger than L2)",
+        "us_per_call": ms * 1e3,
+        "l2": "16 state sets in rotation (201 MB, larger than L2); a CUDA graph of 16 calls replayed",
         "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": st_bytes,
                      "achieved": st_bytes / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": st_bytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,

@@ -62,7 +62,7 @@ constexpr int kMaxPer = 2048;         // positions per attend CTA in the window 
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct Params {
-    int B, n, ns, N_max, H_q, H_kv, group, H_I, M, phi;
+    int B, n, ns, N_max, H_q, H_kv, group, H_I, H_Ik, M, phi;
     int S1, KPC;        // scan CTAs per sequence, keys per scan CTA
     int S2, per;        // attend CTAs per sequence, selected positions per attend CTA
     int window;         // 1: the sparse branch attends over the last M positions (no indexer)
@@ -201,6 +201,57 @@ __device__ void linear_slice(const Params& P, int b, int g, int c0, float* s_sli
     group_sync(kLaBar, kLaThreads);
 }
 
+// One box of the paper's indexer form (a key per indexer head, H_I = 8): 16
+// positions of 8 key rows each (128-byte rows, 128-byte swizzle).  Lane l
+// takes head l / 4 and dims 16 (l % 4) .. + 16; the head's dot product is
+// summed over its 4 lanes, ReLU and weight applied, and the heads summed over
+// the warp.  The key of position p comes from k_I_new (not yet in the cache).
+__device__ __forceinline__ void score_box_per_head(const Params& P, int b, int p, int box0, int k1,
+                                                   const uint8_t* tile, uint32_t* srow,
+                                                   unsigned* hist, const uint32_t (&qh)[8],
+                                                   float w_h) {
+    const int lane = threadIdx.x & 31, hh = lane >> 2, part = lane & 3;
+    constexpr int kPb = kScanRows / 8;
+#pragma unroll 4
+    for (int sp = 0; sp < kPb; ++sp) {
+        const int pos = box0 + sp;
+        const int row = sp * 8 + hh;
+        uint4 u0, u1;
+        if (pos == p) {
+            const uint4* src = reinterpret_cast<const uint4*>(P.k_I_new + ((int64_t)b * 8 + hh) * kDI +
+                                                              16 * part);
+            u0 = src[0];
+            u1 = src[1];
+        } else {
+            const uint8_t* rp = tile + row * 128;
+            const int sw = row & 7;
+            u0 = *reinterpret_cast<const uint4*>(rp + (((2 * part) ^ sw) << 4));
+            u1 = *reinterpret_cast<const uint4*>(rp + (((2 * part + 1) ^ sw) << 4));
+        }
+        const uint32_t kw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[i]));
+            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qh[i]));
+            acc0 = fmaf(kf.x, qf.x, acc0);
+            acc1 = fmaf(kf.y, qf.y, acc1);
+        }
+        float dot = acc0 + acc1;
+        dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+        dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+        float sc = part == 0 ? w_h * fmaxf(dot, 0.0f) : 0.0f;
+        sc += __shfl_xor_sync(0xffffffffu, sc, 4);
+        sc += __shfl_xor_sync(0xffffffffu, sc, 8);
+        sc += __shfl_xor_sync(0xffffffffu, sc, 16);
+        if (lane == 0 && pos < k1) {
+            const uint32_t kk = order_key(sc);
+            srow[pos] = kk;
+            atomicAdd(hist + (kk >> 20), 1u);  // a reduction: nothing waits for it
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     k_decode_scan(const __grid_constant__ CUtensorMap tmap_kI, const Params P) {
     extern __shared__ uint8_t smem_raw[];
@@ -223,7 +274,10 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     const int k0 = j * P.KPC;
     const int k1 = min(n, k0 + P.KPC);
     const int nk = P.window ? 0 : max(0, k1 - k0);  // the window step scans nothing
-    const int nst = (nk + kScanRows - 1) / kScanRows;
+    // a box is 128 k_I rows: 128 positions with one key head, 128 / H_I with a
+    // key per indexer head (the paper's form)
+    const int pb = kScanRows / P.H_Ik;
+    const int nst = (nk + pb - 1) / pb;
     bool ok = true;
 
     if (tid == 0) {
@@ -231,8 +285,8 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         ptx::fence_mbar_init();
         for (int st = 0; st < min(nst, kScanStages); ++st) {
             ptx::mbar_arrive_expect_tx(&bars[st], kBoxBytes);
-            ptx::tma_load_2d(ring + st * kBoxBytes, &tmap_kI, 0, b * P.N_max + k0 + st * kScanRows,
-                             &bars[st]);
+            ptx::tma_load_2d(ring + st * kBoxBytes, &tmap_kI, 0,
+                             (b * P.N_max + k0 + st * pb) * P.H_Ik, &bars[st]);
         }
     }
     // prefetch this CTA's first linear-state slice
@@ -278,9 +332,9 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             kd[i] = kn[i];
             vd[i] = vn[i];
         }
-        if (!P.window && tid < kDI / 8) {
-            const uint4* kin = reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * kDI);
-            reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * kDI)[tid] = kin[tid];
+        if (!P.window && tid < P.H_Ik * kDI / 8) {
+            const uint4* kin = reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * P.H_Ik * kDI);
+            reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * P.H_Ik * kDI)[tid] = kin[tid];
         }
     }
 
@@ -307,6 +361,24 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (2 * tq < P.H_I) w_lo = wb[2 * tq];
         if (2 * tq + 1 < P.H_I) w_hi = wb[2 * tq + 1];
     }
+    // the paper's form (a key per indexer head): this lane's 16 query dims of
+    // head lane / 4, and that head's weight
+    uint32_t qh[8];
+    float w_h = 0.0f;
+    if (P.H_Ik > 1) {
+        const int hh = lane >> 2;
+        if (hh < P.H_I) {
+            const uint4* src =
+                reinterpret_cast<const uint4*>(P.q_I + ((int64_t)b * P.H_I + hh) * kDI + 16 * (lane & 3));
+            const uint4 u0 = src[0], u1 = src[1];
+            qh[0] = u0.x; qh[1] = u0.y; qh[2] = u0.z; qh[3] = u0.w;
+            qh[4] = u1.x; qh[5] = u1.y; qh[6] = u1.z; qh[7] = u1.w;
+            w_h = P.w[(int64_t)b * P.H_I + hh];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qh[i] = 0u;
+        }
+    }
     // Warp w owns ring slot w: it scores boxes w, w + 8, ... by itself (8 row
     // tiles of 16 keys each) and re-arms its slot; no barrier joins the scan
     // warps.
@@ -320,7 +392,10 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             if (lane == 0) record_error(P.status, kDevTimeout);
             break;
         }
-        const int box0 = k0 + st * kScanRows;
+        const int box0 = k0 + st * pb;
+        if (P.H_Ik > 1) {
+            score_box_per_head(P, b, p, box0, k1, tile, srow, hist, qh, w_h);
+        } else
 #pragma unroll 2
         for (int rt = 0; rt < kScanRows / 16; ++rt) {
             const int row0 = rt * 16 + gid;
@@ -370,7 +445,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
                 ptx::fence_proxy_async_shared();
                 ptx::mbar_arrive_expect_tx(bar, kBoxBytes);
                 ptx::tma_load_2d(ring + warp * kBoxBytes, &tmap_kI, 0,
-                                 b * P.N_max + k0 + (st + kScanStages) * kScanRows, bar);
+                                 (b * P.N_max + k0 + (st + kScanStages) * pb) * P.H_Ik, bar);
             }
         }
     }
@@ -601,7 +676,7 @@ Plan make_plan(const Shape& s) {
     const int sms = num_sms();
     const int n = s.L;
     pl.S1 = std::max(1, std::min(sms / std::max(1, s.B), (n + 15) / 16));
-    pl.KPC = align_up((n + pl.S1 - 1) / pl.S1, 16);
+    pl.KPC = align_up((n + pl.S1 - 1) / pl.S1, 16);  // a multiple of the positions per box (16 or 128)
     pl.S1 = (n + pl.KPC - 1) / pl.KPC;
     const int cnt = std::min(s.M, n);
     pl.S2 = std::max(1, std::min(sms / std::max(1, s.B), (cnt + 31) / 32));
@@ -634,7 +709,8 @@ size_t fast_decode_ws_bytes(const Shape& s) {
 
 bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool window) {
     if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD) return false;
-    if (!window && (s.d_I != kDI || s.H_Ik != 1 || s.H_I > 8)) return false;
+    if (!window && (s.d_I != kDI || s.H_I > 8)) return false;
+    if (!window && !(s.H_Ik == 1 || (s.H_Ik == 8 && s.H_I == 8))) return false;
     if (s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
     if (s.L < 1 || s.M < 1 || s.B < 1) return false;
     if (window && make_plan(s).per > kMaxPer) return false;
@@ -653,7 +729,7 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     const Plan pl = make_plan(s);
     Params P;
     P.B = s.B; P.n = s.L; P.ns = pl.ns; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv;
-    P.group = s.group; P.H_I = s.H_I; P.M = s.M; P.phi = s.phi;
+    P.group = s.group; P.H_I = s.H_I; P.H_Ik = s.H_Ik; P.M = s.M; P.phi = s.phi;
     P.S1 = pl.S1; P.KPC = pl.KPC; P.S2 = pl.S2; P.per = pl.per; P.window = window ? 1 : 0;
     P.la_slices = s.B * s.H_kv * (kD / kLaCols);
     P.rowbytes = s.H_kv * kD * 2;
@@ -674,7 +750,8 @@ cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
 
     CUtensorMap tmap;
     memset(&tmap, 0, sizeof(tmap));  // unused by the window step (it scans no keys)
-    if (!window && !make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max, kScanRows))
+    if (!window && !make_tmap_bf16_rows(&tmap, a.k_I_cache, kDI, (uint64_t)s.B * s.N_max * s.H_Ik,
+                                        kScanRows))
         return cudaErrorInvalidValue;
 
     static bool attrs_set[64] = {};
