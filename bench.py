@@ -508,6 +508,73 @@ def run_next_rows(args, wl, copies, D, stream):
     return out
 
 
+# ----------------------------------------------------------------------------- channel gate
+def run_gate_channel(args, device, T_prefill=None):
+    """The per-channel gate (Sec. 3.3 Eq. 5) at the 7B width (3584 channels,
+    D_h 3584): the 16384-token prefill on the tensor cores (TFLOP/s) and the
+    8-token decode, which streams W_g once (GB/s).  L2 is flushed before every
+    timed call."""
+    import numpy as np
+    import torch
+
+    from hybrid_linear_top_lightning_b200 import inputs, lisa
+
+    hbm_peak, tc_peak, peak_kind = _peaks()
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for label, wl in (("prefill", inputs.PREFILL_7B), ("decode", inputs.DECODE_7B)):
+        T = wl.n if label == "prefill" else 1
+        if label == "prefill" and T_prefill:
+            T = T_prefill
+        D_h = N = wl.H_q * wl.d
+        gen = inputs.Generator(wl)
+        h = torch.from_numpy(np.stack([gen.hidden(b, 0, T, D_h) for b in range(wl.B)]))
+        h = h.to(torch.bfloat16).to(device)
+        W = torch.from_numpy(gen.gate_weight(D_h)).to(torch.bfloat16).to(device)
+        o_lin = torch.from_numpy(np.stack([gen.branch("o_lin", b, 0, T) for b in range(wl.B)]))
+        o_lin = o_lin.to(torch.bfloat16).to(device)
+        o_sp = torch.from_numpy(np.stack([gen.branch("o_sp", b, 0, T) for b in range(wl.B)]))
+        o_sp = o_sp.to(torch.bfloat16).to(device)
+        o = torch.empty_like(o_lin)
+        D = lisa.make_dims(wl.B, T, 0, T, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M)
+        ws = lisa.workspace(D, lisa.LISA_OP_GATE_CHANNEL, device)
+        for _ in range(args.warmup):
+            lisa.lisa_gate_channel(D, D_h, h, W, o_lin, o_sp, o, ws, stream)
+        torch.cuda.synchronize()
+        reps = max(3, min(args.steps, 20))
+        tot = 0.0
+        for _ in range(reps):
+            flush.fill_(1)  # evict the previous call's data from L2
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            lisa.lisa_gate_channel(D, D_h, h, W, o_lin, o_sp, o, ws, stream)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            tot += a_.elapsed_time(b_)
+        assert lisa.lisa_check_status(ws, stream) == lisa.LISA_OK
+        ms = tot / reps
+        tokens = wl.B * T
+        nbytes = 2 * (tokens * D_h + N * D_h + 3 * tokens * N)
+        flops = 2.0 * tokens * N * D_h
+        if label == "prefill":
+            roof = {"bound": "tensor", "algorithmic_flops_per_launch": flops,
+                    "achieved": flops / (ms / 1e3) / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": flops / (ms / 1e3) / 1e12 / tc_peak, "peak_kind": peak_kind,
+                    "traffic": None}
+        else:
+            roof = {"bound": "hbm", "algorithmic_bytes_per_launch": nbytes,
+                    "achieved": nbytes / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": nbytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                    "traffic": None}
+        out[label] = {"tokens": tokens, "channels": N, "D_h": D_h, "us_per_call": ms * 1e3,
+                      "value": tokens / (ms / 1e3), "unit": "tok/s", "roofline": roof}
+        del h, W, o_lin, o_sp, o, ws
+    out["what"] = ("per-channel gate g = sigmoid(W_g h) mixing the branches (Eq. 5): "
+                   "lisa_gate_channel, 7B width")
+    return out
+
+
 # ----------------------------------------------------------------------------- prefill
 def prefill_work(wl) -> dict:
     """Algorithmic work of one causal prefill of wl.n tokens per sequence: causal
@@ -673,6 +740,10 @@ def main():
                     help="prefill length of the prefill line (default: the 7B workload's 16384)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill line and print it (for profiling runs)")
+    ap.add_argument("--gate-only", action="store_true",
+                    help="time only the per-channel gate lines and print them (for profiling)")
+    ap.add_argument("--gate-T", type=int, default=0,
+                    help="prefill tokens of the channel-gate line (default: 16384)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -706,7 +777,14 @@ def main():
             if rank == 0:
                 print(json.dumps({"prefill": run_prefill(args, wl_p, device)}), flush=True)
             return
+        if args.gate_only:
+            if rank == 0:
+                print(json.dumps({"gate_channel": run_gate_channel(args, device, args.gate_T)}),
+                      flush=True)
+            return
         line = run_gpu(args, wl, rank, world, device)
+        if args.next_rows:
+            line["gate_channel"] = run_gate_channel(args, device)
         if args.prefill_steps > 0:
             line["prefill"] = run_prefill(args, wl_p, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -120,6 +120,7 @@ size_t workspace_bytes(const Shape& s, int op) {
             return need > fast ? need : fast;
         }
         case LISA_OP_PREFILL: return prefill_ws(s).end;
+        case LISA_OP_GATE_CHANNEL: return kStatusBytes;
         default: return 0;
     }
 }
@@ -146,7 +147,7 @@ extern "C" {
 lisa_status lisa_workspace_size(const lisa_dims* dims, int op, size_t* bytes) {
     LISA_TRY(check_dims(dims));
     if (!bytes) return LISA_ERR_INVALID_ARG;
-    if (op < LISA_OP_TOPM || op > LISA_OP_PREFILL) return LISA_ERR_INVALID_ARG;
+    if (op < LISA_OP_TOPM || op > LISA_OP_GATE_CHANNEL) return LISA_ERR_INVALID_ARG;
     *bytes = workspace_bytes(resolve(*dims), op);
     return LISA_OK;
 }
@@ -357,6 +358,21 @@ lisa_status lisa_state_transfer(const lisa_dims* dims, float* S, float* S_start,
     if ((int64_t)s.B * s.H_kv == 0) return LISA_OK;
     if (!S || !S_start || !grad_sum) return LISA_ERR_INVALID_ARG;
     return cuda_status(state_transfer(s, S, S_start, grad_sum, t, alpha, (cudaStream_t)stream));
+}
+
+lisa_status lisa_gate_channel(const lisa_dims* dims, int32_t D_h, const void* h, const void* W_g,
+                              const void* o_lin, const void* o_sparse, void* o, void* ws,
+                              size_t ws_bytes, void* stream) {
+    LISA_TRY(check_dims(dims));
+    if (D_h < 1) return LISA_ERR_INVALID_ARG;
+    const Shape s = resolve(*dims);
+    if ((int64_t)s.B * s.T == 0) return LISA_OK;
+    if (!h || !W_g || !o_lin || !o_sparse || !o) return LISA_ERR_INVALID_ARG;
+    LISA_TRY(check_ws(ws, ws_bytes, kStatusBytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (fast_gate_channel_supported(s, D_h, h, W_g, o_lin, o_sparse, o))
+        return cuda_status(fast_gate_channel(s, D_h, h, W_g, o_lin, o_sparse, o, ws, st));
+    return cuda_status(generic_gate_channel(s, D_h, h, W_g, o_lin, o_sparse, o, st));
 }
 
 lisa_status lisa_check_status(void* ws, void* stream) {

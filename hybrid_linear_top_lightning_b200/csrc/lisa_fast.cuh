@@ -47,4 +47,14 @@ cudaError_t fast_gate(const Shape& s, const void* logit, const void* o_lin, cons
 cudaError_t state_transfer(const Shape& s, float* S, float* S_start, float* grad_sum, int t,
                            float alpha, cudaStream_t st);
 
+
+// gate_channel.cu: per-channel gate (Sec. 3.3 Eq. 5), bf16, N % 256 == 0, D_h % 64 == 0
+bool fast_gate_channel_supported(const Shape& s, int D_h, const void* h, const void* W,
+                                 const void* o_lin, const void* o_sp, const void* o);
+cudaError_t generic_gate_channel(const Shape& s, int D_h, const void* h, const void* W,
+                                 const void* o_lin, const void* o_sp, void* o, cudaStream_t st);
+cudaError_t fast_gate_channel(const Shape& s, int D_h, const void* h, const void* W,
+                              const void* o_lin, const void* o_sp, void* o, void* ws,
+                              cudaStream_t st);
+
 }  // namespace lisa

@@ -44,4 +44,19 @@ inline bool make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A 2-D bf16 tensor [rows][inner] read in boxes of box_inner x box_rows with the
+// 128-byte swizzle (box_inner * 2 must be 128).
+inline bool make_tmap_bf16_box(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                               uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn fn = tma_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace lisa

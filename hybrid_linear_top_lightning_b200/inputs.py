@@ -16,6 +16,9 @@ evaluates; the values are synthetic):
 * ``q, k, v, q_I, k_I`` ~ N(0, sigma^2) per coordinate.  ``sigma`` is 1 for
   the tiny fp32 workload and 1/sqrt(128) for the model-shaped workloads.
 * ``w`` (indexer head weights) ~ U(0, 1); ``gate`` (gate logits) ~ N(0, 1).
+* Per-channel gate inputs: hidden states ``h`` [B, n, D_h] ~ N(0, 1); gate
+  weights ``W_g`` [H_q*d, D_h] ~ N(0, 1/D_h), so a gate logit is ~ N(0, 1);
+  branch outputs ``o_lin``, ``o_sp`` [B, n, H_q, d] ~ N(0, 1).
 * Planted heavy keys: per batch element, floor(0.01 * n) positions drawn
   uniformly without replacement among the n positions of the workload; at
   each, ``3 * sigma * sqrt(dim) * u`` is added to ``k`` (every KV head) and to
@@ -38,6 +41,7 @@ BLOCK = 1024  # positions per random stream block
 _TENSOR_IDS = {
     "q": 1, "k": 2, "v": 3, "q_I": 4, "k_I": 5, "w": 6, "gate": 7,
     "plant": 8, "u_k": 9, "u_kI": 10, "qL": 11, "kL": 12, "vL": 13,
+    "h": 14, "W_g": 15, "o_lin": 16, "o_sp": 17,
 }
 
 
@@ -195,6 +199,22 @@ class Generator:
         """Gate logits of the linear branch, one per (position, query head)."""
         x = self._per_position("gate", b, p0, p1, self.wl.H_q, "normal", 1.0)
         return self._finish(x)
+
+    def hidden(self, b: int, p0: int, p1: int, D_h: int) -> np.ndarray:
+        """Hidden states entering the module, one row of D_h per position."""
+        return self._finish(self._per_position("h", b, p0, p1, D_h, "normal", 1.0))
+
+    def gate_weight(self, D_h: int) -> np.ndarray:
+        """Per-channel gate weights W_g [H_q*d, D_h] (row c feeds channel c)."""
+        N = self.wl.H_q * self.wl.d
+        rng = self._rng("W_g", D_h)
+        x = rng.standard_normal((N, D_h), dtype=np.float32) * np.float32(1.0 / math.sqrt(D_h))
+        return self._finish(x)
+
+    def branch(self, name: str, b: int, p0: int, p1: int) -> np.ndarray:
+        """A branch output ("o_lin" or "o_sp") [p1-p0, H_q, d] for the gate alone."""
+        x = self._per_position(name, b, p0, p1, self.wl.H_q * self.wl.d, "normal", 1.0)
+        return self._finish(x).reshape(p1 - p0, self.wl.H_q, self.wl.d)
 
     # -- whole-batch helpers -------------------------------------------------
     def batch(self, fn: str, p0: int, p1: int) -> np.ndarray:

@@ -35,6 +35,7 @@ LISA_OP_LINEAR_PREFILL = 2
 LISA_OP_DECODE_STEP = 3
 LISA_OP_DENSE_ATTN = 4
 LISA_OP_PREFILL = 5
+LISA_OP_GATE_CHANNEL = 6
 
 # Every symbol the header declares.
 EXPORTS = (
@@ -42,7 +43,7 @@ EXPORTS = (
     "lisa_linear_decode", "lisa_gate_fuse", "lisa_decode_step", "lisa_dense_attn",
     "lisa_workspace_size", "lisa_check_status", "lisa_status_string", "lisa_version",
     "lisa_topm_noalloc", "lisa_prefill", "lisa_window_indices", "lisa_decode_step_window",
-    "lisa_state_transfer",
+    "lisa_state_transfer", "lisa_gate_channel",
 )
 
 
@@ -111,6 +112,7 @@ def load() -> ctypes.CDLL:
         "lisa_window_indices": [dp, vp, vp, vp],
         "lisa_decode_step_window": [dp, ctypes.POINTER(lisa_decode_args), vp, sz, vp],
         "lisa_state_transfer": [dp, vp, vp, vp, ctypes.c_int32, ctypes.c_float, vp],
+        "lisa_gate_channel": [dp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, sz, vp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -284,3 +286,9 @@ def lisa_check_status(ws, stream=None) -> int:
 
 def default_sm_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def lisa_gate_channel(dims, D_h: int, h, W_g, o_lin, o_sparse, o, ws, stream=None):
+    _check(load().lisa_gate_channel(ctypes.byref(dims), int(D_h), _ptr(h), _ptr(W_g), _ptr(o_lin),
+                                    _ptr(o_sparse), _ptr(o), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "lisa_gate_channel")

@@ -110,7 +110,8 @@ typedef enum lisa_op {
     LISA_OP_LINEAR_PREFILL = 2,
     LISA_OP_DECODE_STEP = 3,
     LISA_OP_DENSE_ATTN = 4,
-    LISA_OP_PREFILL = 5
+    LISA_OP_PREFILL = 5,
+    LISA_OP_GATE_CHANNEL = 6
 } lisa_op;
 
 /* Lightning Indexer scores (Sec. 3.2; the per-head score vector defined under
@@ -254,6 +255,24 @@ LISA_API lisa_status lisa_decode_step_window(const lisa_dims* dims, const lisa_d
  * Errors: LISA_ERR_INVALID_ARG for t < 1, a NaN alpha or a null pointer. */
 LISA_API lisa_status lisa_state_transfer(const lisa_dims* dims, float* S, float* S_start,
                                          float* grad_sum, int32_t t, float alpha, void* stream);
+
+/* Per-channel gate (LISA Sec. 3.3, Eq. 5) joining the branches as in Eq. 1:
+ *   g[m][c] = sigmoid(sum_k W_g[c][k] h[m][k]),
+ *   o[m][c] = g o_lin[m][c] + (1 - g) o_sparse[m][c]
+ * for every token m of the B*T tokens and channel c of the H_q*d output
+ * channels (query head major).  Device arrays of the activation type:
+ * h [B,T,D_h] (the module's input hidden states), W_g [H_q*d, D_h] (row c is
+ * channel c's gate weights), o_lin, o_sparse, o [B,T,H_q,d].  Nothing is
+ * retained; o may alias neither input.  On bf16 with H_q*d a multiple of 256,
+ * D_h a multiple of 64 and 16-byte aligned arrays the contraction runs on the
+ * tensor cores (tiles of 128 tokens; fewer than 64 tokens take a kernel that
+ * streams W_g once); every other size takes a plain kernel.
+ * Workspace: lisa_workspace_size(.., LISA_OP_GATE_CHANNEL) (the status word).
+ * Errors: LISA_ERR_INVALID_ARG for D_h < 1 or a null pointer; a device wait
+ * that gives up is reported by lisa_check_status as LISA_ERR_TIMEOUT. */
+LISA_API lisa_status lisa_gate_channel(const lisa_dims* dims, int32_t D_h, const void* h,
+                                       const void* W_g, const void* o_lin, const void* o_sparse,
+                                       void* o, void* ws, size_t ws_bytes, void* stream);
 
 /* Dense causal softmax attention over every cached position s <= p (Sec. 3.1,
  * the standard attention LISA replaces); the O(n) reference line. */

@@ -42,3 +42,21 @@ def test_host_validation_without_gpu():
     # null pointers are rejected before launch
     st = lisa.load().lisa_gate_fuse(ctypes.byref(good), None, None, None, None, None)
     assert st == lisa.LISA_ERR_INVALID_ARG
+
+
+def test_every_operation_has_a_workspace_size():
+    """Each LISA_OP_* the header declares answers lisa_workspace_size; one past
+    the last is rejected."""
+    src = open(os.path.join(ROOT, "include", "lisa.h")).read()
+    ops = {k: int(v) for k, v in re.findall(r"\b(LISA_OP_\w+)\s*=\s*(\d+)", src)}
+    assert ops and sorted(ops.values()) == list(range(len(ops)))
+    good = lisa.make_dims(8, 1, 16383, 16384, 28, 4, 128, 8, 1, 64, 2048)
+    for name, op in ops.items():
+        assert getattr(lisa, name) == op, name
+        assert lisa.lisa_workspace_size(good, op) > 0, name
+    n = ctypes.c_size_t(0)
+    st = lisa.load().lisa_workspace_size(ctypes.byref(good), len(ops), ctypes.byref(n))
+    assert st == lisa.LISA_ERR_INVALID_ARG
+    st = lisa.load().lisa_gate_channel(ctypes.byref(good), 0, None, None, None, None, None, None,
+                                       0, None)
+    assert st == lisa.LISA_ERR_INVALID_ARG
