@@ -513,7 +513,8 @@ def run_gate_channel(args, device, T_prefill=None):
     """The per-channel gate (Sec. 3.3 Eq. 5) at the 7B width (3584 channels,
     D_h 3584): the 16384-token prefill on the tensor cores (TFLOP/s) and the
     8-token decode, which streams W_g once (GB/s).  L2 is flushed before every
-    timed call."""
+    timed prefill call; the decode calls rotate over copies of W_g larger than
+    L2 together."""
     import numpy as np
     import torch
 
@@ -542,18 +543,39 @@ def run_gate_channel(args, device, T_prefill=None):
         for _ in range(args.warmup):
             lisa.lisa_gate_channel(D, D_h, h, W, o_lin, o_sp, o, ws, stream)
         torch.cuda.synchronize()
-        reps = max(3, min(args.steps, 20))
-        tot = 0.0
-        for _ in range(reps):
-            flush.fill_(1)  # evict the previous call's data from L2
+        if label == "prefill":
+            reps = max(3, min(args.steps, 20))
+            tot = 0.0
+            for _ in range(reps):
+                flush.fill_(1)  # evict the previous call's data from L2
+                a_ = torch.cuda.Event(enable_timing=True)
+                b_ = torch.cuda.Event(enable_timing=True)
+                a_.record(stream)
+                lisa.lisa_gate_channel(D, D_h, h, W, o_lin, o_sp, o, ws, stream)
+                b_.record(stream)
+                torch.cuda.synchronize()
+                tot += a_.elapsed_time(b_)
+            ms = tot / reps
+        else:
+            # a call is a few microseconds, shorter than a host launch: one graph of
+            # 8 calls over 8 copies of W_g (207 MB in rotation, larger than L2)
+            Ws = [W] + [W.clone() for _ in range(7)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for Wc in Ws:
+                    lisa.lisa_gate_channel(D, D_h, h, Wc, o_lin, o_sp, o, ws)
+            g.replay()
+            torch.cuda.synchronize()
+            reps = max(4, args.steps // 4)
             a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a_.record(stream)
-            lisa.lisa_gate_channel(D, D_h, h, W, o_lin, o_sp, o, ws, stream)
+            for _ in range(reps):
+                g.replay()
             b_.record(stream)
             torch.cuda.synchronize()
-            tot += a_.elapsed_time(b_)
+            ms = a_.elapsed_time(b_) / (reps * len(Ws))
+            del g, Ws
         assert lisa.lisa_check_status(ws, stream) == lisa.LISA_OK
-        ms = tot / reps
         tokens = wl.B * T
         nbytes = 2 * (tokens * D_h + N * D_h + 3 * tokens * N)
         flops = 2.0 * tokens * N * D_h

@@ -235,20 +235,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
 }
 
 // Up to 64 tokens (decode): W_g streamed from HBM once, on the warp MMA.
-// A CTA owns 16 channels; its 8 warps split K in 32-column chunks (warp w takes
-// chunks w, w+8, ...).  Per chunk a lane reads 16 bytes of W_g row g and of row
+// A CTA owns 16 channels; its warps split K in 32-column chunks (warp w of WN
+// takes chunks w, w+WN, ...).  Per chunk a lane reads 16 bytes of W_g row g and of row
 // g+8 (g = lane/4, t = lane%4: columns 8t..8t+7 of the chunk) and 16 bytes of
 // token g's h at the same columns.  The 32 columns are fed to two m16n8k16
 // MMAs in a column order that A and B share (MMA j takes columns 8t+4j..8t+4j+3
 // of lane (g, t) as its k = 2t, 2t+1, 2t+8, 2t+9), which leaves the sum over k
 // unchanged, so neither operand needs shared memory.  NT tiles of 8 tokens.
-constexpr int kRowWarps = 8;
+template <int NT>
+struct RowCfg {
+    // warps per CTA and chunks in flight per warp: at D_h = 3584 (112 chunks)
+    // one token tile reads its whole W_g share in a single round of loads
+    static constexpr int warps = NT <= 2 ? 16 : 8;
+    static constexpr int unroll = NT == 1 ? 7 : NT == 2 ? 4 : NT == 4 ? 4 : 2;
+};
 
 template <int NT>
-__global__ void __launch_bounds__(kRowWarps * 32) k_gate_channel_rows(
+__global__ void __launch_bounds__(RowCfg<NT>::warps * 32) k_gate_channel_rows(
     const bf16* __restrict__ h, const bf16* __restrict__ W, int M, int N, int K,
     const bf16* __restrict__ o_lin, const bf16* __restrict__ o_sp, bf16* __restrict__ o) {
-    constexpr int kRowUnroll = NT >= 4 ? 2 : 4;  // chunks in flight per warp
+    constexpr int kRowWarps = RowCfg<NT>::warps;
+    constexpr int kRowUnroll = RowCfg<NT>::unroll;
     __shared__ float red[kRowWarps][NT][16][8];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) k_gate_channel_rows(
 template <int NT>
 void launch_rows(int M, int N, int K, const void* h, const void* W, const void* o_lin,
                  const void* o_sp, void* o, cudaStream_t st) {
-    k_gate_channel_rows<NT><<<N / 16, kRowWarps * 32, 0, st>>>(
+    k_gate_channel_rows<NT><<<N / 16, RowCfg<NT>::warps * 32, 0, st>>>(
         (const bf16*)h, (const bf16*)W, M, N, K, (const bf16*)o_lin, (const bf16*)o_sp, (bf16*)o);
 }
 

@@ -33,6 +33,15 @@ MUTANTS = {
                      "g * o_sp[base + c] + (1.0 - g) * o_lin[base + c]"),
     "elu_shift_dropped": ("return x > 0.0 ? x + 1.0 : std::exp(x);", "return x > 0.0 ? x : std::exp(x);"),
     "softmax_max_wrong": ("const double e = std::exp(logit[i] - mx);", "const double e = std::exp(logit[i]);"),
+    "window_short": ("const int first = std::max(0, p - D->M + 1);",
+                     "const int first = std::max(0, p - D->M + 2);"),
+    "transfer_mean_over_t": ("grad_sum[i] / (t - 1)", "grad_sum[i] / t"),
+    "transfer_alpha_swapped": ("(1.0 - alpha) * grad_t + alpha * mean_prev",
+                               "alpha * grad_t + (1.0 - alpha) * mean_prev"),
+    "transfer_start_kept": ("        S_start[i] = S_t;\n", "        S_start[i] = S_start[i];\n"),
+    "channel_gate_swapped": ("(1.0 - g) * o_sp[base + c] + g * o_lin[base + c]",
+                             "g * o_sp[base + c] + (1.0 - g) * o_lin[base + c]"),
+    "channel_weight_transposed": ("W_g[(int64_t)c * D_h + k]", "W_g[(int64_t)k * N + c]"),
 }
 
 
@@ -46,7 +55,8 @@ def _run_mutant(name, old, new, tmp):
                    check=True)
     env = dict(os.environ, LISA_REF_LIB=mlib, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle.py")],
+                        os.path.join(ROOT, "tests", "test_oracle.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_next.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     return name, r.returncode
 
