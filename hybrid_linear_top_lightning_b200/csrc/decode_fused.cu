@@ -13,8 +13,8 @@
 //    ring slot w and scores whole boxes on the tensor cores (mma m16n8k16:
 //    keys x indexer heads, K = d_I), then ReLU, head weights and head sum.
 //    The order-preserving keys of the scores go to a workspace row, and each
-//    key's top 12 bits are counted into the sequence's histogram (global
-//    reductions issued as the keys are made).
+//    key's top 12 bits are counted in a shared-memory histogram of the CTA,
+//    added to the sequence's histogram once the CTA's keys are done.
 //    Linear-branch warps (concurrently): one slice (sequence, KV head, 32
 //    value columns) of S += phi(k)^T v and o_lin = phi(q) S (/ phi(q).z).
 //    CTA 0 of each sequence appends the new k, v, k_I to the caches.
@@ -119,7 +119,8 @@ struct ScanSmem {
     static constexpr int zloc = vcol + kLaCols * 4;                  // float[128]
     static constexpr int den = zloc + kD * 4;                        // float[16]
     static constexpr int bars = den + 16 * 4;                        // uint64[kScanStages]
-    static constexpr int total = bars + kScanStages * 8 + 1024;      // + base alignment slack
+    static constexpr int shist = bars + kScanStages * 8;             // u32[4096] key histogram
+    static constexpr int total = shist + 4096 * 4 + 1024;            // + base alignment slack
 };
 
 // One slice of the linear branch: sequence b, KV head g, value columns [c0, c0+32).
@@ -247,7 +248,7 @@ __device__ __forceinline__ void score_box_per_head(const Params& P, int b, int p
         if (lane == 0 && pos < k1) {
             const uint32_t kk = order_key(sc);
             srow[pos] = kk;
-            atomicAdd(hist + (kk >> 20), 1u);  // a reduction: nothing waits for it
+            atomicAdd(hist + (kk >> 20), 1u);  // the CTA's shared-memory histogram
         }
     }
 }
@@ -265,8 +266,10 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
     float* zloc = reinterpret_cast<float*>(base + ScanSmem::zloc);
     float* den = reinterpret_cast<float*>(base + ScanSmem::den);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + ScanSmem::bars);
+    unsigned* shist = reinterpret_cast<unsigned*>(base + ScanSmem::shist);
 
     ptx::pdl_launch_dependents();
+    for (int i = threadIdx.x; i < 4096; i += blockDim.x) shist[i] = 0u;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
     const int b = blockIdx.x / P.S1, j = blockIdx.x % P.S1;
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         }
         const int box0 = k0 + st * pb;
         if (P.H_Ik > 1) {
-            score_box_per_head(P, b, p, box0, k1, tile, srow, hist, qh, w_h);
+            score_box_per_head(P, b, p, box0, k1, tile, srow, shist, qh, w_h);
         } else
 #pragma unroll 2
         for (int rt = 0; rt < kScanRows / 16; ++rt) {
@@ -435,7 +438,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             if (tq < 2 && pos < k1) {
                 const uint32_t kk = order_key(tq == 0 ? s0 : s1);
                 srow[pos] = kk;
-                atomicAdd(hist + (kk >> 20), 1u);  // a reduction: nothing waits for it
+                atomicAdd(shist + (kk >> 20), 1u);
             }
         }
         if (st + kScanStages < nst) {
@@ -448,6 +451,14 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
                                  (b * P.N_max + k0 + (st + kScanStages) * pb) * P.H_Ik, bar);
             }
         }
+    }
+    // the CTA's key histogram joins the sequence's: one reduction per non-empty
+    // bin (the keys of a row crowd into few bins, so per-key global atomics
+    // would queue on the same addresses)
+    group_sync(kScanBar, kScanThreads);
+    for (int i = tid; i < 4096; i += kScanThreads) {
+        const unsigned c = shist[i];
+        if (c) atomicAdd(hist + i, c);
     }
     if (!ok && lane == 0) {
         // give this warp's copy still in flight a bounded chance to land before exit

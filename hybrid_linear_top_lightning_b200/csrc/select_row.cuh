@@ -20,7 +20,8 @@
 //     its rank in position order (ties go to the lowest positions); a block
 //     scan of the selected counts gives each thread the rank of its first
 //     selected position; threads whose ranks meet [lo, hi) rebuild bit masks
-//     of their chunk and write out[rank - lo] = position.
+//     of their chunk and write out[rank - lo] = position (in one round through
+//     shared memory, so that the index row leaves in coalesced stores).
 #pragma once
 
 #include "lisa_internal.cuh"
@@ -34,6 +35,10 @@ struct SelectSmem {
     unsigned* hist;   // 4096 u32
     int* bc;          // >= 64 ints: broadcasts and scan scratch
     uint2* cand;      // kCandTotal (key, position)
+    // the candidate buffer once the ranks are known: the index row is
+    // scattered here by rank and leaves in coalesced stores
+    __device__ int* stage() const { return reinterpret_cast<int*>(cand); }
+    static constexpr int kStageCap = kCandTotal * 2;
 };
 
 // Exclusive block scan of v; `total` gets the block sum.  Two barriers: the
@@ -298,9 +303,31 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
     }
     const uint32_t tau = prefix;  // the M-th largest key; krem of its ties are kept
 
-    // emits this thread's selected positions of round r with ranks in [lo, hi);
-    // `keep` = how many of its keys equal to tau are kept (its lowest ones)
-    auto emit = [&](int r, int rank, int keep) {
+    // emits this thread's selected positions of round r with ranks in [lo, hi)
+    // to dst[rank - lo]; `keep` = how many of its keys equal to tau are kept
+    // (its lowest ones)
+    auto emit = [&](int* dst, int r, int rank, int keep) {
+        if (REG) {
+            // the thread's keys are in registers in position order: one pass
+            int eq_seen = 0;
+#pragma unroll
+            for (int j = 0; j < kQ; ++j) {
+                uint32_t k[4];
+                const int q = word(r, j, k);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool v = 4 * q + e < n;
+                    const bool eq = v && k[e] == tau;
+                    const bool take = (v && k[e] > tau) || (eq && eq_seen < keep);
+                    eq_seen += eq;
+                    if (take) {
+                        if (rank >= lo && rank < hi) dst[rank - lo] = 4 * q + e;
+                        ++rank;
+                    }
+                }
+            }
+            return;
+        }
         uint64_t gtm = 0, eqm = 0;
 #pragma unroll
         for (int j = 0; j < kQ; ++j) {
@@ -323,7 +350,7 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
         while (m) {
             const int b = __ffsll((long long)m) - 1;
             m &= m - 1;
-            if (rank >= lo && rank < hi) out[rank - lo] = pos0 + b;
+            if (rank >= lo && rank < hi) dst[rank - lo] = pos0 + b;
             ++rank;
         }
     };
@@ -346,8 +373,17 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
         }
         const int sel_t = above + gt_c + keep;
         int sel_tot;
+        // the scan's barriers also end every read of the candidate buffer
         const int rank = sel_block_excl_scan<NT>(sel_t, bc + 32, sel_tot);
-        if (rank < hi && rank + sel_t > lo) emit(0, rank, keep);
+        const int nout = min(hi, sel_tot) - lo;
+        if (nout > SelectSmem::kStageCap) {
+            if (rank < hi && rank + sel_t > lo) emit(out, 0, rank, keep);
+        } else if (nout > 0) {
+            int* stage = sm.stage();
+            if (rank < hi && rank + sel_t > lo) emit(stage, 0, rank, keep);
+            __syncthreads();
+            for (int i = tid; i < nout; i += NT) out[i] = stage[i];
+        }
         __syncthreads();
         return;
     }
@@ -381,7 +417,7 @@ __device__ void row_topm(const uint32_t* row, bool resident, int n, int M, const
         int sel_tot;
         const int rank = rank_base + sel_block_excl_scan<NT>(sel_t, bc + 32, sel_tot);
         rank_base += sel_tot;
-        if (rank < hi && rank + sel_t > lo) emit(r, rank, keep);
+        if (rank < hi && rank + sel_t > lo) emit(out, r, rank, keep);
     }
     __syncthreads();
 }
