@@ -42,6 +42,7 @@
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
 #include "attend_core.cuh"
+#include "decode_linear.cuh"
 #include "select_row.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
@@ -57,7 +58,7 @@ constexpr int kScanThreads = 256;
 constexpr int kScanRows = 128;        // keys per TMA box (16 per warp)
 constexpr int kScanStages = 8;        // boxes in flight per CTA
 constexpr int kBoxBytes = kScanRows * kDI * 2;
-constexpr int kLaCols = 32;           // linear-state columns per slice
+constexpr int kLaCols = dec::kLaCols;  // linear-state columns per slice
 constexpr int kMaxPer = 2048;         // positions per attend CTA in the window step
 constexpr uint32_t kWaitTries = 1u << 22;
 
@@ -97,17 +98,11 @@ struct Params {
 
 __host__ __device__ inline int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
-constexpr int kLaThreads = 128;       // linear-branch warps of the scan kernel
-constexpr int kScanBar = 1, kLaBar = 2;  // named barriers of the two warp groups
-
-__device__ __forceinline__ void group_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ float feat(int phi, float x) {
-    if (phi == LISA_PHI_IDENTITY) return x;
-    return x > 0.0f ? x + 1.0f : __expf(x);
-}
+using dec::kLaThreads;
+using dec::kLaBar;
+using dec::group_sync;
+using dec::feat;
+constexpr int kScanBar = 1;  // named barrier of the scan warps (the linear-branch warps use kLaBar)
 
 // ============================================================================ K1: scan
 struct ScanSmem {
@@ -122,85 +117,6 @@ struct ScanSmem {
     static constexpr int shist = bars + kScanStages * 8;             // u32[4096] key histogram
     static constexpr int total = shist + 4096 * 4 + 1024;            // + base alignment slack
 };
-
-// One slice of the linear branch: sequence b, KV head g, value columns [c0, c0+32).
-// s_slice holds S[:, c0:c0+32] of that head (already loaded).  Run by the
-// kLaThreads threads that follow the scan threads of the block.
-__device__ void linear_slice(const Params& P, int b, int g, int c0, float* s_slice, float* fk,
-                             float* fq, float* vcol, float* zloc, float* den) {
-    const int tid = threadIdx.x - kScanThreads, lane = tid & 31, warp = tid >> 5;
-    const bf16* kl = P.k_L + ((int64_t)b * P.H_kv + g) * kD;
-    const bf16* vl = P.v_L + ((int64_t)b * P.H_kv + g) * kD;
-    // 128-bit loads: 8 bf16 per load, one load per thread for each vector
-    auto unpack8 = [](const uint4& u, float (&f)[8]) {
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 t = __bfloat1622float2(h2[e]);
-            f[2 * e] = t.x;
-            f[2 * e + 1] = t.y;
-        }
-    };
-    for (int e = tid; e < kD / 8 + kLaCols / 8 + P.group * (kD / 8); e += kLaThreads) {
-        float f[8];
-        if (e < kD / 8) {
-            unpack8(reinterpret_cast<const uint4*>(kl)[e], f);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) fk[8 * e + x] = feat(P.phi, f[x]);
-        } else if (e < kD / 8 + kLaCols / 8) {
-            const int e2 = e - kD / 8;
-            unpack8(reinterpret_cast<const uint4*>(vl + c0)[e2], f);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) vcol[8 * e2 + x] = f[x];
-        } else {
-            const int e3 = e - kD / 8 - kLaCols / 8;
-            const int h = e3 / (kD / 8), c8 = e3 % (kD / 8);
-            unpack8(reinterpret_cast<const uint4*>(
-                        P.q_L + ((int64_t)b * P.H_q + g * P.group + h) * kD)[c8], f);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) fq[h * kD + 8 * c8 + x] = feat(P.phi, f[x]);
-        }
-    }
-    ptx::cp_async_wait_all();  // the state slice (when it was prefetched)
-    group_sync(kLaBar, kLaThreads);
-    const bool norm = P.phi == LISA_PHI_ELU1_NORM;
-    float* Sg = P.S + ((int64_t)b * P.H_kv + g) * kD * kD;
-    if (norm) {
-        const float* zg = P.z + ((int64_t)b * P.H_kv + g) * kD;
-        for (int i = tid; i < kD; i += kLaThreads) zloc[i] = zg[i] + fk[i];
-    }
-    for (int e = tid; e < kD * kLaCols; e += kLaThreads) {
-        const int i = e / kLaCols, c = e % kLaCols;
-        const float nv = fmaf(fk[i], vcol[c], s_slice[e]);
-        s_slice[e] = nv;
-        Sg[(int64_t)i * kD + c0 + c] = nv;
-    }
-    group_sync(kLaBar, kLaThreads);
-    if (norm) {
-        // z itself is advanced by the attend kernel: the sibling slices of this
-        // head still read the old z here
-        for (int h = warp; h < P.group; h += kLaThreads / 32) {
-            float dz = 0.0f;
-            for (int i = lane; i < kD; i += 32) dz = fmaf(fq[h * kD + i], zloc[i], dz);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) dz += __shfl_xor_sync(0xffffffffu, dz, o);
-            if (lane == 0) den[h] = dz;
-        }
-        group_sync(kLaBar, kLaThreads);
-    }
-    for (int e = tid; e < P.group * kLaCols; e += kLaThreads) {
-        const int h = e / kLaCols, c = e % kLaCols;
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four independent chains
-#pragma unroll 8
-        for (int i = 0; i < kD; i += 4)
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                acc[u] = fmaf(fq[h * kD + i + u], s_slice[(i + u) * kLaCols + c], acc[u]);
-        const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        P.olin[((int64_t)b * P.H_q + g * P.group + h) * kD + c0 + c] = norm ? sum / den[h] : sum;
-    }
-    group_sync(kLaBar, kLaThreads);
-}
 
 // One box of the paper's indexer form (a key per indexer head, H_I = 8): 16
 // positions of 8 key rows each (128-byte rows, 128-byte swizzle).  Lane l
@@ -311,7 +227,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
         if (slice < P.la_slices) {
             const int lb = slice / slices_per_b, lg = (slice / (kD / kLaCols)) % P.H_kv;
             const int lc0 = (slice % (kD / kLaCols)) * kLaCols;
-            linear_slice(P, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
+            dec::linear_slice(P, kScanThreads, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
         }
         for (int sl = slice + gridDim.x; sl < P.la_slices; sl += gridDim.x) {
             const int lb = sl / slices_per_b, lg = (sl / (kD / kLaCols)) % P.H_kv;
@@ -320,7 +236,7 @@ __global__ void __launch_bounds__(kScanThreads + kLaThreads, 1)
             for (int e = tid - kScanThreads; e < kD * kLaCols; e += kLaThreads)
                 s_slice[e] = Sg[(int64_t)(e / kLaCols) * kD + lc0 + e % kLaCols];
             group_sync(kLaBar, kLaThreads);
-            linear_slice(P, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
+            dec::linear_slice(P, kScanThreads, lb, lg, lc0, s_slice, fk, fq, vcol, zloc, den);
         }
         return;
     }
@@ -694,7 +610,7 @@ Plan make_plan(const Shape& s) {
     pl.per = (cnt + pl.S2 - 1) / pl.S2;
     pl.S2 = (cnt + pl.per - 1) / pl.per;
     pl.ns = align_up(n, 32);
-    size_t off = kStatusBytes;
+    size_t off = decode_scratch_offset(s.B);
     auto take = [&](size_t bytes) {
         const size_t at = off;
         off += (bytes + 255) & ~(size_t)255;
@@ -703,7 +619,7 @@ Plan make_plan(const Shape& s) {
     pl.scores = take(sizeof(uint32_t) * (size_t)s.B * pl.ns);
     pl.olin = take(sizeof(float) * (size_t)s.B * s.H_q * kD);
     pl.part = take(sizeof(float) * (size_t)s.B * pl.S2 * s.H_q * (kD + 2));
-    pl.hist = take(sizeof(unsigned) * (size_t)s.B * 4096);
+    pl.hist = decode_hist_offset();
     pl.sel = take(sizeof(int32_t) * (size_t)s.B * s.M);
     pl.end = off;
     return pl;
@@ -715,7 +631,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 size_t fast_decode_ws_bytes(const Shape& s) {
     if (s.B <= 0 || s.L <= 0) return kStatusBytes;
-    return make_plan(s).end;
+    return std::max(make_plan(s).end, coop_decode_ws_bytes(s));
 }
 
 bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool window) {
@@ -737,6 +653,7 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool windo
 
 cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
                              bool window) {
+    if (!window && coop_decode_supported(s, a)) return coop_decode_step(s, a, ws, st);
     const Plan pl = make_plan(s);
     Params P;
     P.B = s.B; P.n = s.L; P.ns = pl.ns; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv;

@@ -60,7 +60,7 @@ TopmWs topm_ws(const Shape& s) {
 struct DecodeWs { size_t scores, idx, count, o_sp, o_lin, end; };
 DecodeWs decode_ws(const Shape& s) {
     DecodeWs w;
-    w.scores = kStatusBytes;
+    w.scores = decode_scratch_offset(s.B);  // after the state the fast paths keep between calls
     w.idx = w.scores + align256(sizeof(float) * (size_t)s.B * s.L);
     w.count = w.idx + align256(sizeof(int32_t) * (size_t)s.B * s.M);
     w.o_sp = w.count + align256(sizeof(int32_t) * (size_t)s.B);

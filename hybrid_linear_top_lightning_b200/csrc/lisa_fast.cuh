@@ -7,12 +7,24 @@
 
 namespace lisa {
 
-// Fused decode step (decode_fused.cu).
+// Decode-step workspaces start with state that is zero between calls, at
+// offsets that depend on B only, so that one workspace serves a batch at every
+// context length: [status | key histograms, B x 4096 u32 | barrier lines,
+// B x 128 bytes | scratch of the call].
+inline size_t decode_hist_offset() { return kStatusBytes; }
+inline size_t decode_sync_offset(int B) { return kStatusBytes + (size_t)B * 4096 * 4; }
+inline size_t decode_scratch_offset(int B) { return decode_sync_offset(B) + (size_t)B * 128; }
+
+// Decode step: one cooperative kernel over all SMs (decode_coop.cu) when it
+// covers the call, else the four-kernel form (decode_fused.cu).
 size_t fast_decode_ws_bytes(const Shape& s);
 // window: the sparse branch attends over the last M positions (no indexer)
 bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool window = false);
 cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
                              bool window = false);
+size_t coop_decode_ws_bytes(const Shape& s);
+bool coop_decode_supported(const Shape& s, const lisa_decode_args& a);
+cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st);
 
 // Top-M over many query rows (prefill).
 size_t fast_topm_ws_bytes(const Shape& s);

@@ -48,7 +48,11 @@
  *    bytes of device memory, 256-byte aligned, ZERO-FILLED ONCE when allocated;
  *    the library keeps the first 256 bytes (status word) and re-initialises the
  *    rest itself.  A workspace must not be shared by calls that may run
- *    concurrently.
+ *    concurrently.  The decode steps keep state between calls in the workspace
+ *    (key histograms and exchange counters, all zero again when a call ends) at
+ *    offsets that depend on B only: one workspace, sized for the largest
+ *    context, serves a batch as its context grows; zero-fill it again after B
+ *    changes or after lisa_check_status has returned LISA_ERR_TIMEOUT.
  */
 #ifndef LISA_H_
 #define LISA_H_
