@@ -127,6 +127,74 @@ __device__ __forceinline__ void attn_issue_stage(uint8_t* ring, int* spos, int c
     }
 }
 
+// One stage of 16 keys for one warp (the bulk-copy gathers of the decode and
+// prefill kernels): K rows at shared address kb, V rows at vb, `krow` bytes
+// apart, the warp's KV head `head_off` bytes into each row; qf are its query
+// fragments (the layout of AttQ).  Key k of the stage counts iff bit k of
+// `valid` is set (each lane reads bits gid and gid + 8).  Updates the warp's
+// online-softmax state: m and l (base 2; l summed over this lane's keys only)
+// and o, in the layout of AttOut.
+__device__ __forceinline__ void attn_stage16(const uint32_t (&qf)[8][2], uint32_t kb, uint32_t vb,
+                                             int krow, uint32_t head_off, unsigned valid,
+                                             float scale_log2, float (&m)[2], float (&l)[2],
+                                             float (&o)[8][4]) {
+    const int lane = threadIdx.x & 31, gid = lane >> 2;
+    // ldmatrix lane addressing: K as A (keys x dims), V as A^T (dims x keys)
+    const int ka_key = (lane & 7) + ((lane >> 3) & 1) * 8, ka_dim = (lane >> 4) * 8;
+    const int va_key = (lane & 7) + (lane >> 4) * 8, va_dim = ((lane >> 3) & 1) * 8;
+    float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ks += 2) {
+        uint32_t a0[4], a1[4];
+        ptx::ldmatrix_x4(a0, kb + ka_key * krow + head_off + (ks * 16 + ka_dim) * 2);
+        ptx::ldmatrix_x4(a1, kb + ka_key * krow + head_off + ((ks + 1) * 16 + ka_dim) * 2);
+        ptx::mma_bf16(s0, a0, qf[ks][0], qf[ks][1]);
+        ptx::mma_bf16(s1, a1, qf[ks + 1][0], qf[ks + 1][1]);
+    }
+    // element e: key gid + 8 (e >> 1), head slot 2tq + (e & 1)
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const bool ok = (valid >> (gid + 8 * r)) & 1u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            v[2 * r + h] = ok ? (s0[2 * r + h] + s1[2 * r + h]) * scale_log2 : -INFINITY;
+    }
+    float corr[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float mt = fmaxf(v[h], v[2 + h]);
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        const float m_new = fmaxf(m[h], mt);
+        corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m[h] - m_new);
+        m[h] = m_new;
+        l[h] *= corr[h];
+    }
+    float pr[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float mm = m[e & 1];
+        pr[e] = (mm == -INFINITY) ? 0.0f : exp2f(v[e] - mm);
+        l[e & 1] += pr[e];
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        o[t][0] *= corr[0]; o[t][1] *= corr[1];
+        o[t][2] *= corr[0]; o[t][3] *= corr[1];
+    }
+    // P^T fragments (keys x heads) -> B operand (k = keys, n = heads)
+    const uint32_t b0 = ptx::movmatrix_trans(ptx::pack_bf16(pr[0], pr[1]));
+    const uint32_t b1 = ptx::movmatrix_trans(ptx::pack_bf16(pr[2], pr[3]));
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        uint32_t va[4];
+        ptx::ldmatrix_x4_trans(va, vb + va_key * krow + head_off + (t * 16 + va_dim) * 2);
+        ptx::mma_bf16(o[t], va, b0, b1);
+    }
+}
+
 // q: the row's query fragments (attn_load_q), `group` <= 8 heads per KV
 // head.  pos[0..cnt): positions (shared or global memory), gathered from
 // `src`; positions outside [0, src.p_max] are masked out and reported through

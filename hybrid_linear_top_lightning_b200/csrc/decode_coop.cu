@@ -46,10 +46,10 @@
 
 #include <algorithm>
 
+#include "attend_core.cuh"
 #include "decode_linear.cuh"
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
-#include "select_row.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
 
@@ -616,9 +616,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 4; ++e) o[t][e] = 0.0f;
         const uint32_t head_off = (uint32_t)(g * kD * 2);
         const int krow = P.krow;
-        // ldmatrix lane addressing: K as A (keys x dims), V as A^T (dims x keys)
-        const int ka_key = (lane & 7) + ((lane >> 3) & 1) * 8, ka_dim = (lane >> 4) * 8;
-        const int va_key = (lane & 7) + (lane >> 4) * 8, va_dim = ((lane >> 3) & 1) * 8;
         // stages below `known` positions exist; past it, the count is final once
         // the refinement has reported
         int known = def_full;
@@ -642,58 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const uint32_t kb = ptx::smem_u32(ring + slot * P.stage_bytes);
-            const uint32_t vb = kb + kGK * krow;
-            float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int ks = 0; ks < 8; ks += 2) {
-                uint32_t a0[4], a1[4];
-                ptx::ldmatrix_x4(a0, kb + ka_key * krow + head_off + (ks * 16 + ka_dim) * 2);
-                ptx::ldmatrix_x4(a1, kb + ka_key * krow + head_off + ((ks + 1) * 16 + ka_dim) * 2);
-                ptx::mma_bf16(s0, a0, qf[ks][0], qf[ks][1]);
-                ptx::mma_bf16(s1, a1, qf[ks + 1][0], qf[ks + 1][1]);
-            }
-            // element e: key gid + 8 (e >> 1), head slot 2tq + (e & 1)
-            float v[4];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const bool listed = st * kGK + gid + 8 * r < known;
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    v[2 * r + h] = listed ? (s0[2 * r + h] + s1[2 * r + h]) * P.scale_log2 : -INFINITY;
-            }
-            float corr[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float mt = fmaxf(v[h], v[2 + h]);
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                const float m_new = fmaxf(m[h], mt);
-                corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m[h] - m_new);
-                m[h] = m_new;
-                l[h] *= corr[h];
-            }
-            float pr[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float mm = m[e & 1];
-                pr[e] = (mm == -INFINITY) ? 0.0f : exp2f(v[e] - mm);
-                l[e & 1] += pr[e];
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                o[t][0] *= corr[0]; o[t][1] *= corr[1];
-                o[t][2] *= corr[0]; o[t][3] *= corr[1];
-            }
-            // P^T fragments (keys x heads) -> B operand (k = keys, n = heads)
-            const uint32_t b0 = ptx::movmatrix_trans(ptx::pack_bf16(pr[0], pr[1]));
-            const uint32_t b1 = ptx::movmatrix_trans(ptx::pack_bf16(pr[2], pr[3]));
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                uint32_t va[4];
-                ptx::ldmatrix_x4_trans(va, vb + va_key * krow + head_off + (t * 16 + va_dim) * 2);
-                ptx::mma_bf16(o[t], va, b0, b1);
-            }
+            const int left = known - st * kGK;  // keys of this stage in the list
+            attn_stage16(qf, kb, kb + kGK * krow, krow, head_off,
+                         left >= kGK ? 0xFFFFu : (1u << left) - 1u, P.scale_log2, m, l, o);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&empty[slot]);
         }

@@ -22,13 +22,16 @@ def _dv(a, dt=BF):
     return torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
 
 
-def run_decode_case(wl, phi=0, zero_qI=False, S0_from_prefill=True, check_state=True):
+def run_decode_case(wl, phi=0, zero_qI=False, S0_from_prefill=True, check_state=True,
+                    kI_first_half_scale=1.0):
     """One decode step at position n-1 over a cache of n-1 tokens; returns errors."""
     gen = inputs.Generator(wl)
     n, p, B = wl.n, wl.n - 1, wl.B
     kc_np = gen.batch("k", 0, n)
     vc_np = gen.batch("v", 0, n)
     kI_np = gen.batch("k_I", 0, n)
+    # a power of two keeps the bf16 values exact on both sides
+    kI_np[:, : n // 2] *= kI_first_half_scale
     q = gen.batch("q", p, n)
     q_I = gen.batch("q_I", p, n)
     if zero_qI:
@@ -124,3 +127,11 @@ def test_decode_fused_matches_generic_path_outputs_shape():
     a = run_decode_case(wl)
     b = run_decode_case(wl)
     np.testing.assert_array_equal(a["idx"], b["idx"])
+
+
+def test_decode_scores_skewed_across_the_context():
+    """Indexer keys 4x larger in the first half of the context: the top-M comes
+    almost entirely from there, so the parts of the context whose own scores
+    suggest a lower threshold have to contribute through the exact path too."""
+    res = run_decode_case(inputs.DECODE_7B.with_(B=2, n=16384, M=2048), kI_first_half_scale=4.0)
+    assert np.all(res["cnt"] == 2048)
