@@ -73,9 +73,9 @@ def decode_bytes(wl) -> dict:
                 total=per_seq * wl.B)
 
 
-DECODE_KERNELS_PER_STEP = 4  # scan, select, attend, combine
-DECODE_SOURCES = ("decode_fused.cu", "attend_core.cuh", "select_row.cuh", "sm100_ptx.cuh",
-                  "tma_host.cuh", "lisa_internal.cuh")
+DECODE_KERNELS_PER_STEP = 1  # k_decode_coop: the whole step in one cooperative launch
+DECODE_SOURCES = ("decode_coop.cu", "attend_core.cuh", "decode_linear.cuh", "sm100_ptx.cuh",
+                  "tma_host.cuh", "lisa_internal.cuh", "lisa_fast.cuh")
 
 
 def _kernel_source_hash() -> str:
@@ -89,9 +89,10 @@ def _kernel_source_hash() -> str:
 
 
 def _profiled_traffic(wl):
-    """DRAM bytes of one decode step (its four kernels) from the committed ncu
-    summary, if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", "decode_fused_traffic.json")
+    """DRAM bytes of one decode step (one k_decode_coop launch) from the
+    committed ncu summary, if it was taken on the current kernel sources; else
+    None."""
+    path = os.path.join(ROOT, "profiles", "decode_coop_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
@@ -344,7 +345,7 @@ def run_gpu(args, wl, rank, world, device):
                          f"(caches, state, inputs) used in rotation, "
                          f"{args.rotate} x {bytes_['total'] / 1e6:.1f} MB touched per cycle",
                    "step": "decode step: append, linear update+readout, indexer scan, "
-                           "top-M, sparse attention, gate (4 kernels, PDL-chained)",
+                           "top-M, sparse attention, gate (one cooperative kernel)",
                    "launch": "CUDA graph replay of lisa_decode_step" if args.graphs
                              else "lisa_decode_step from the host"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -352,9 +353,8 @@ def run_gpu(args, wl, rank, world, device):
                      "frac_of_8TBs": achieved / 8000.0,
                      "traffic": _profiled_traffic(wl),
                      "algorithmic_bytes_per_launch": bytes_["total"],
-                     "kernel": "decode step: one lisa_decode_step call = k_decode_scan + "
-                               "k_decode_select + k_decode_attend + k_decode_combine "
-                               "(PDL-chained)",
+                     "kernel": "decode step: one lisa_decode_step call = one k_decode_coop "
+                               "launch (cooperative, one CTA per SM)",
                      "launch_us": avg_s * 1e6},
         "e2e": {"value": job_throughput(B, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
