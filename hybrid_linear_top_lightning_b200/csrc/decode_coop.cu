@@ -99,6 +99,7 @@ static_assert(8 * 36 * 32 * 4 <= kCandOff, "softmax-state exchange below the can
 
 struct CoopParams {
     int B, n, N_max, H_q, H_kv, group, H_I, H_Ik, M, phi;
+    int window;         // 1: the Stage-1 step, attending over the last M positions (no indexer)
     int ncta, KPC;      // CTAs per sequence, positions per CTA
     int nstg;           // gather stages in the ring
     int rowbytes;       // bytes of one cached K (or V) row: H_kv * kD * 2
@@ -359,10 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gid = lane >> 2, tq = lane & 3;
     const int b = blockIdx.x / P.ncta, j = blockIdx.x % P.ncta;
     const int n = P.n, p = n - 1;
-    const int k0 = j * P.KPC;
+    // the positions the CTAs of a sequence share out: all n, or the window's last min(M, n)
+    const int first = P.window ? n - min(P.M, n) : 0;
+    const int k0 = first + j * P.KPC;
     const int k1 = min(n, k0 + P.KPC);
     const int nk = max(0, k1 - k0);
-    const bool sel_all = n <= P.M;  // every position is kept: no scores needed
+    const bool sel_all = P.window || n <= P.M;  // every position is kept: no scores needed
     unsigned* sync = P.sync + (int64_t)b * 32;
 
     for (int i = tid; i < 4096; i += kThreads) shist[i] = 0u;
@@ -411,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kd[i] = kn[i];
                 vd[i] = vn[i];
             }
-            if (tid < P.H_Ik * kDI / 8) {
+            if (!P.window && tid < P.H_Ik * kDI / 8) {
                 const uint4* kin = reinterpret_cast<const uint4*>(P.k_I_new + (int64_t)b * P.H_Ik * kDI);
                 reinterpret_cast<uint4*>(P.k_I_cache + ((int64_t)b * P.N_max + p) * P.H_Ik * kDI)[tid] =
                     kin[tid];
@@ -422,7 +425,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t qb[8], qh[8];
         float w_lo = 0.0f, w_hi = 0.0f, w_h = 0.0f;
         const float* wb = P.w + (int64_t)b * P.H_I;
-        if (P.H_Ik == 1) {
+        if (sel_all) {
+            // nothing to score (the window step's indexer inputs may be null)
+        } else if (P.H_Ik == 1) {
             if (gid < P.H_I) {
                 const uint4* src =
                     reinterpret_cast<const uint4*>(P.q_I + ((int64_t)b * P.H_I + gid) * kDI + 16 * tq);
@@ -1018,10 +1023,10 @@ struct CoopPlan {
     bool fits;
 };
 
-CoopPlan coop_plan(const Shape& s) {
+CoopPlan coop_plan(const Shape& s, bool window) {
     CoopPlan pl;
     const int sms = coop_num_sms();
-    const int n = s.L;
+    const int n = window ? std::min(s.M, s.L) : s.L;  // positions shared out over the CTAs
     const int per_b = sms / std::max(1, s.B);
     pl.ncta = std::max(1, std::min(per_b, (n + 15) / 16));
     pl.KPC = align_up((n + pl.ncta - 1) / pl.ncta, 16);
@@ -1030,7 +1035,7 @@ CoopPlan coop_plan(const Shape& s) {
     pl.stage_bytes = 2 * kGK * pl.krow;
     pl.nstg = std::min(kMaxStages, kCandOff / pl.stage_bytes);
     pl.sel_cap = std::min(pl.KPC, s.M);
-    pl.ns = align_up(n, 32);
+    pl.ns = align_up(s.L, 32);
     pl.spos_off = kKeysOff + align_up(4 * pl.KPC, 128);
     pl.smem = pl.spos_off + align_up(4 * pl.sel_cap, 128) + 1024;  // + base alignment slack
     size_t off = decode_scratch_offset(s.B);
@@ -1055,29 +1060,32 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 size_t coop_decode_ws_bytes(const Shape& s) {
     if (s.B <= 0 || s.L <= 0) return kStatusBytes;
-    return coop_plan(s).end;
+    return std::max(coop_plan(s, false).end, coop_plan(s, true).end);
 }
 
-bool coop_decode_supported(const Shape& s, const lisa_decode_args& a) {
-    if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD || s.d_I != kDI || s.H_I > 8) return false;
-    if (!(s.H_Ik == 1 || (s.H_Ik == 8 && s.H_I == 8))) return false;
+bool coop_decode_supported(const Shape& s, const lisa_decode_args& a, bool window) {
+    if (s.dtype != LISA_BF16 || s.T != 1 || s.d != kD) return false;
+    if (!window && (s.d_I != kDI || s.H_I > 8 || !(s.H_Ik == 1 || (s.H_Ik == 8 && s.H_I == 8))))
+        return false;
     if (s.group > 8 || !(s.H_kv == 1 || s.H_kv == 2 || s.H_kv == 4)) return false;
     if (s.L < 1 || s.M < 1 || s.B < 1) return false;
-    if (!coop_plan(s).fits) return false;
-    const void* ptrs[] = {a.q,       a.k_new,   a.v_new, a.q_L,     a.k_L,   a.v_L,
-                          a.k_cache, a.v_cache, a.S,     a.o,       a.q_I,   a.k_I_new,
-                          a.k_I_cache};
+    if (!coop_plan(s, window).fits) return false;
+    const void* ptrs[] = {a.q, a.k_new, a.v_new, a.q_L, a.k_L, a.v_L, a.k_cache, a.v_cache, a.S, a.o};
     for (const void* p : ptrs)
         if (!aligned16(p)) return false;
+    if (!window && (!aligned16(a.q_I) || !aligned16(a.k_I_new) || !aligned16(a.k_I_cache)))
+        return false;
     if (s.phi == LISA_PHI_ELU1_NORM && !aligned16(a.z)) return false;
-    return tma_encode_fn() != nullptr;
+    return window || tma_encode_fn() != nullptr;
 }
 
-cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st) {
-    const CoopPlan pl = coop_plan(s);
+cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
+                             bool window) {
+    const CoopPlan pl = coop_plan(s, window);
     CoopParams P;
     P.B = s.B; P.n = s.L; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv; P.group = s.group;
     P.H_I = s.H_I; P.H_Ik = s.H_Ik; P.M = s.M; P.phi = s.phi;
+    P.window = window ? 1 : 0;
     P.ncta = pl.ncta; P.KPC = pl.KPC; P.nstg = pl.nstg;
     P.rowbytes = s.H_kv * kD * 2; P.krow = pl.krow; P.stage_bytes = pl.stage_bytes;
     P.sel_cap = pl.sel_cap; P.ns = pl.ns; P.spos_off = pl.spos_off;
@@ -1097,10 +1105,12 @@ cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     P.cand = (uint2*)(w8 + pl.cand);
     P.gsel = (int*)(w8 + pl.gsel);
 
-    CUtensorMap tmap_slot, tmap_tail;
+    CUtensorMap tmap_slot, tmap_tail;  // unused by the window step (it scans no keys)
+    memset(&tmap_slot, 0, sizeof(tmap_slot));
+    memset(&tmap_tail, 0, sizeof(tmap_tail));
     const uint64_t kI_rows = (uint64_t)s.B * s.N_max * s.H_Ik;
-    if (!make_tmap_bf16_rows(&tmap_slot, a.k_I_cache, kDI, kI_rows, kSlotRows) ||
-        !make_tmap_bf16_rows(&tmap_tail, a.k_I_cache, kDI, kI_rows, kBoxRows))
+    if (!window && (!make_tmap_bf16_rows(&tmap_slot, a.k_I_cache, kDI, kI_rows, kSlotRows) ||
+                    !make_tmap_bf16_rows(&tmap_tail, a.k_I_cache, kDI, kI_rows, kBoxRows)))
         return cudaErrorInvalidValue;
 
     static bool attr_set[64] = {};

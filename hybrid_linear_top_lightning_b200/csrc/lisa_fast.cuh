@@ -23,8 +23,9 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool windo
 cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
                              bool window = false);
 size_t coop_decode_ws_bytes(const Shape& s);
-bool coop_decode_supported(const Shape& s, const lisa_decode_args& a);
-cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st);
+bool coop_decode_supported(const Shape& s, const lisa_decode_args& a, bool window);
+cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
+                             bool window);
 
 // Top-M over many query rows (prefill).
 size_t fast_topm_ws_bytes(const Shape& s);
