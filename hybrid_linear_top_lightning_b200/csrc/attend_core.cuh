@@ -103,10 +103,15 @@ __device__ __forceinline__ int attn_stage_pos(const int* pos, int cnt, int st) {
 }
 
 // Issues this thread's 16-byte asynchronous copies of stage st into ring slot
-// st % kAttStages and records the stage's positions (-1 past the list).
-template <int HKV>
+// st % kAttStages and records the stage's positions (-1 past the list).  With
+// SPLIT, the K row of each key instead goes by one 1-D bulk copy (from the
+// key's first thread, arriving on kbar[slot]) and the threads copy the V rows
+// only: the two copy paths of the SM share the gather (on the 7B prefill,
+// 8.1 ms against 8.7 ms with 16-byte copies alone; 3/4 of K by bulk copy was
+// no better than none).
+template <int HKV, bool SPLIT = false>
 __device__ __forceinline__ void attn_issue_stage(uint8_t* ring, int* spos, int cnt, int st, int raw,
-                                                 const AttSrc& src) {
+                                                 const AttSrc& src, uint64_t* kbar = nullptr) {
     using A = AttGeo<HKV>;
     using bf16 = __nv_bfloat16;
     constexpr int GK = A::keys;
@@ -117,6 +122,21 @@ __device__ __forceinline__ void attn_issue_stage(uint8_t* ring, int* spos, int c
     const int ps = (raw < 0 || raw > src.p_max) ? 0 : raw;  // never dereference out of range
     const bf16* ksrc = (ps == src.p_special) ? src.k_special : src.k_cache + (src.row0 + ps) * kb_row;
     const bf16* vsrc = (ps == src.p_special) ? src.v_special : src.v_cache + (src.row0 + ps) * kb_row;
+    if (SPLIT) {
+        if (sub == 0) {
+            uint64_t* bar = kbar + st % kAttStages;
+            ptx::fence_proxy_async_shared();  // the slot's earlier reads precede the copy
+            ptx::mbar_arrive_expect_tx(bar, A::rowbytes);
+            ptx::bulk_load(dst + ck * A::krow, ksrc, A::rowbytes, bar);
+        }
+#pragma unroll
+        for (int u = 0; u < A::cpt / 2; ++u) {
+            const int off = sub + u * A::tpk;
+            ptx::cp_async_16(dst + GK * A::krow + ck * A::krow + off * 16,
+                             reinterpret_cast<const uint4*>(vsrc) + off);
+        }
+        return;
+    }
 #pragma unroll
     for (int u = 0; u < A::cpt; ++u) {
         const int i = sub + u * A::tpk;
@@ -201,10 +221,10 @@ __device__ __forceinline__ void attn_stage16(const uint32_t (&qf)[8][2], uint32_
 // `status`.  `ring` holds AttGeo<HKV>::ring_bytes bytes, `spos` (shared
 // memory) kAttStages * AttGeo<HKV>::keys ints; both are clobbered.  The
 // result is valid in the warps with part == 0 (warp % wph == 0).
-template <int HKV>
+template <int HKV, bool SPLIT = false>
 __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spos, const int* pos,
                                           int cnt, const AttSrc& src, float scale_log2,
-                                          unsigned* status, AttOut& out) {
+                                          unsigned* status, AttOut& out, uint64_t* kbar = nullptr) {
     using A = AttGeo<HKV>;
     constexpr int GK = A::keys;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -214,7 +234,13 @@ __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spo
     const int nst = (cnt + GK - 1) / GK;
     const int p_max = src.p_max;
     auto load_pos = [&](int st) { return attn_stage_pos<HKV>(pos, cnt, st); };
-    auto issue_stage = [&](int st, int raw) { attn_issue_stage<HKV>(ring, spos, cnt, st, raw, src); };
+    auto issue_stage = [&](int st, int raw) {
+        attn_issue_stage<HKV, SPLIT>(ring, spos, cnt, st, raw, src, kbar);
+    };
+    if (SPLIT && tid == 0) {
+        for (int i = 0; i < kAttStages; ++i) ptx::mbar_init(kbar + i, GK);  // one arrival per key
+        ptx::fence_mbar_init();
+    }
 
     float* m = out.m;  // heads 2tq, 2tq + 1
     float* l = out.l;
@@ -242,6 +268,8 @@ __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spo
 #pragma unroll 1
     for (int st = 0; st < nst; ++st) {
         ptx::cp_async_wait_group<kAttStages - 2>();  // this thread's copies of stage st landed
+        if (SPLIT && !ptx::mbar_wait_bounded(kbar + st % kAttStages, (st / kAttStages) & 1, 1u << 22))
+            record_error(status, kDevTimeout);  // (the stage's K rows)
         // all copies of stage st are visible, and every warp is done with
         // stage st - 1, whose slot the next issue reuses
         __syncthreads();

@@ -1,7 +1,8 @@
 // Sparse softmax attention over given index lists (lisa_sparse_attn) for many
-// query rows, bf16, head dim 128: one CTA per query row runs the gather and
-// tensor-core online softmax of attend_core.cuh over the row's count[b,t]
-// positions and writes the normalised output (LISA, arXiv 2607.19358v1,
+// query rows, bf16, head dim 128: one CTA per query row runs the gather (K rows
+// by 1-D bulk copies, V rows by 16-byte cp.async) and tensor-core online
+// softmax of attend_core.cuh over the row's count[b,t] positions and writes
+// the normalised output (LISA, arXiv 2607.19358v1,
 // Sec. 3.2 Eq. 1, the SA_M branch).  Positions outside [0, p] are masked out
 // and reported as LISA_ERR_DEVICE_BOUNDS through the status word.
 #include "attend_core.cuh"
@@ -28,7 +29,8 @@ template <int HKV>
 struct SpSmem {
     static constexpr int spos = 0;                                     // int[stages][keys]
     static constexpr int ring = (kAttStages * AttGeo<HKV>::keys * 4 + 127) / 128 * 128;
-    static constexpr int total = ring + AttGeo<HKV>::ring_bytes;
+    static constexpr int kbar = ring + AttGeo<HKV>::ring_bytes;        // uint64[kAttStages]
+    static constexpr int total = kbar + kAttStages * 8;
     static_assert(total <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -45,7 +47,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) k_sparse_rows(const SpParams P
     const AttQ q = attn_load_q<HKV>(P.q + (int64_t)row * P.H_q * 128, P.group);
     AttOut r;
     const AttSrc kv{P.k, P.v, (int64_t)b * P.N_max, p, -1, nullptr, nullptr};
-    attn_core<HKV>(q, sp_raw + L::ring, spos, pos, cnt, kv, P.scale_log2, P.status, r);
+    attn_core<HKV, true>(q, sp_raw + L::ring, spos, pos, cnt, kv, P.scale_log2, P.status, r,
+                         reinterpret_cast<uint64_t*>(sp_raw + L::kbar));
     // normalised output of each KV head's query heads (group rows of 128 dims,
     // contiguous in o), staged by the head's first warp in its own slot of the
     // ring and stored with 16-byte writes
