@@ -72,17 +72,18 @@ constexpr int kBoxRows = 16;             // rows per TMA box
 constexpr int kBoxBytes = kBoxRows * kDI * 2;
 constexpr int kGK = 16;                  // keys per gather stage
 constexpr int kMaxStages = 16;
-// The ring holds the scan slots and the linear-branch buffers in phase A, the
-// candidates in phase B, the gather stages in phase C and the exchange of
-// softmax states at the end of C.
-constexpr int kLaOff = kSlots * kSlotBytes;
-constexpr int kLaBytes = kD * kLaCols * 4 + kD * 4 + 8 * kD * 4 + kLaCols * 4 + kD * 4 + 16 * 4;
+// The ring holds the scan slots in phase A, the gather stages in phase C and
+// the exchange of softmax states at the end of C.
 constexpr int kRingBytes = 163 * 1024;
-// Candidates of the threshold digit, kept in the ring's top while the gather
-// stages fill the rest (4 stages of 16 keys at 4 KV heads).
+// The ring's top: the linear-branch buffers in phase A, then the candidates of
+// the threshold digit (both used by warps 8-11 only); the gather stages (4 of 16
+// keys at 4 KV heads) stay below it, so the attention warps can fill them while
+// the linear branch still runs.
 constexpr int kCandBytes = 32 * 1024;
 constexpr int kCandOff = kRingBytes - kCandBytes;
 constexpr int kCandSmem = kCandBytes / 8;
+constexpr int kLaOff = kCandOff;
+constexpr int kLaBytes = kD * kLaCols * 4 + kD * 4 + 8 * kD * 4 + kLaCols * 4 + kD * 4 + 16 * 4;
 constexpr int kHistOff = kRingBytes;                 // u32[4096]
 constexpr int kBarOff = kHistOff + 4096 * 4;         // mbarriers: full[16], empty[16], scan[8]
 constexpr int kMiscOff = kBarOff + 512;              // int[128]
@@ -94,7 +95,8 @@ constexpr int kRefFirst = kMainThreads + 32;
 constexpr int kRefThreads = kThreads - kRefFirst;
 constexpr uint32_t kWaitTries = 1u << 22;
 constexpr uint32_t kSpinTries = 1u << 20;
-static_assert(kLaOff + kLaBytes <= kRingBytes, "linear-branch buffers beside the scan slots");
+static_assert(kLaOff + kLaBytes <= kRingBytes && kSlots * kSlotBytes <= kLaOff,
+              "linear-branch buffers above the scan slots and the gather stages");
 static_assert(8 * 36 * 32 * 4 <= kCandOff, "softmax-state exchange below the candidates");
 
 struct CoopParams {
@@ -625,6 +627,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the refinement has reported
         int known = def_full;
         bool fin = sel_all;
+        // This warp fetches the V bytes it alone reads (its KV head's 256 bytes
+        // of each V row of its stages) with 16-byte cp.async copies, one own stage
+        // ahead; the K rows come by the gather warp's bulk copies.  A slot is
+        // reused every nstg stages, a multiple of NG, so the V bytes a warp
+        // overwrites are ones it has read itself.
+        const int64_t rowel = (int64_t)P.H_kv * kD;
+        const bf16* vsrc0 = P.v_cache + (int64_t)b * P.N_max * rowel + g * kD;
+        const bf16* vnew = P.v_new + (int64_t)b * rowel + g * kD;
+        const int ahead = P.nstg / NG - 1;  // own stages of V in flight beyond the current one
+        int v_next = qg;                    // the next own stage whose V is not requested yet
+        auto request_v = [&](int s) {
+            const int nin = min(kGK, known - s * kGK);
+            uint8_t* vdst = ring + (s % P.nstg) * P.stage_bytes + kGK * krow + g * kD * 2;
+#pragma unroll
+            for (int u = 0; u < kGK * 16 / 32; ++u) {
+                const int c = lane + 32 * u, key = c >> 4, off = c & 15;
+                const int pos = spos[s * kGK + min(key, nin - 1)];
+                const bf16* src = pos == p ? vnew : vsrc0 + pos * rowel;
+                ptx::cp_async_16(vdst + key * krow + off * 16, reinterpret_cast<const uint4*>(src) + off);
+            }
+            ptx::cp_async_commit();
+        };
 #pragma unroll 1
         for (int st = qg;; st += NG) {
             if (st * kGK >= known) {
@@ -638,6 +662,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (st * kGK >= known) break;
             }
+            while (v_next <= st + NG * ahead && v_next * kGK < known) {
+                request_v(v_next);
+                v_next += NG;
+            }
+            if (v_next > st + NG)
+                ptx::cp_async_wait_group<1>();  // this stage's V landed (the next one may not have)
+            else
+                ptx::cp_async_wait_group<0>();
+            __syncwarp();
             const int slot = st % P.nstg;
             if (!ptx::mbar_wait_bounded(&full[slot], (st / P.nstg) & 1, kWaitTries)) {
                 if (lane == 0) record_error(P.status, kDevTimeout);
@@ -658,6 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the warps of a KV head hand their states to warp g (the ring is free
         // once every attention warp is past its last stage)
+        ptx::cp_async_wait_all();  // (V copies requested for stages past a timeout)
         group_sync(kConsBar, kMainThreads);
         float* xf = reinterpret_cast<float*>(ring) + warp * 36 * 32 + lane;  // [36][32] per warp
         if (qg != 0) {
@@ -705,13 +739,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 8) {
-        // producer: the K and V rows of stage st, key i by lanes i (K) and 16 + i (V);
-        // a short last stage repeats its first position (those keys are masked)
+        // producer: the K rows of stage st by 1-D bulk copies, key i by lane i (the
+        // attention warps fetch the V rows); a short last stage repeats its first
+        // position (those keys are masked)
         const int64_t rowel = (int64_t)P.H_kv * kD;
         const bf16* kn = P.k_new + (int64_t)b * rowel;
-        const bf16* vn = P.v_new + (int64_t)b * rowel;
-        const int kk = lane & (kGK - 1);
-        const bool isv = lane >= kGK;
         int issued = 0;
         bool ok = ptx::mbar_wait_bounded(def_ready, 0, kWaitTries);
         if (!ok && lane == 0) record_error(P.status, kDevTimeout);
@@ -741,14 +773,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::fence_proxy_async_shared();
             }
             uint8_t* dst = ring + slot * P.stage_bytes;
-            if (lane == 0) ptx::mbar_arrive_expect_tx(&full[slot], 2u * kGK * (uint32_t)P.rowbytes);
+            if (lane == 0) ptx::mbar_arrive_expect_tx(&full[slot], kGK * (uint32_t)P.rowbytes);
             __syncwarp();
             const int nin = min(kGK, known - st * kGK);
-            const int pos = spos[st * kGK + min(kk, nin - 1)];
-            const bf16* src = pos == p ? (isv ? vn : kn)
-                                       : (isv ? P.v_cache : P.k_cache) + ((int64_t)b * P.N_max + pos) * rowel;
-            ptx::bulk_load(dst + (isv ? kGK * P.krow : 0) + kk * P.krow, src, (uint32_t)P.rowbytes,
-                           &full[slot]);
+            if (lane < kGK) {
+                const int pos = spos[st * kGK + min(lane, nin - 1)];
+                const bf16* src = pos == p ? kn : P.k_cache + ((int64_t)b * P.N_max + pos) * rowel;
+                ptx::bulk_load(dst + lane * P.krow, src, (uint32_t)P.rowbytes, &full[slot]);
+            }
             issued = st + 1;
         }
         if (!ok) {
@@ -1034,6 +1066,7 @@ CoopPlan coop_plan(const Shape& s, bool window) {
     pl.krow = s.H_kv * kD * 2 + 16;
     pl.stage_bytes = 2 * kGK * pl.krow;
     pl.nstg = std::min(kMaxStages, kCandOff / pl.stage_bytes);
+    pl.nstg -= pl.nstg % (8 / std::max(1, s.H_kv));  // a multiple of the warps per KV head
     pl.sel_cap = std::min(pl.KPC, s.M);
     pl.ns = align_up(s.L, 32);
     pl.spos_off = kKeysOff + align_up(4 * pl.KPC, 128);
