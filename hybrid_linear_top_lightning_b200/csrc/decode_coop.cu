@@ -90,6 +90,7 @@ constexpr int kMiscOff = kBarOff + 512;              // int[128]
 constexpr int kKeysOff = kMiscOff + 512;             // u32[KPC], then int[sel_cap]
 constexpr int kMaxKPC = 8192;
 constexpr int kConsBar = 1;              // named barrier of the attention warps (0-7)
+constexpr int kMiscCBase = 96;    // misc: this CTA's range of the candidate list
 constexpr int kRefBar = 4;               // named barrier of the refinement warps (9-11)
 constexpr int kRefFirst = kMainThreads + 32;
 constexpr int kRefThreads = kThreads - kRefFirst;
@@ -156,6 +157,22 @@ __device__ __forceinline__ void gsync(int bar) {
         asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(NT) : "memory");
 }
 
+// Arrival on counter c (release: this thread's earlier writes, and those
+// ordered before it by a barrier, are visible to whoever acquires the count).
+__device__ __forceinline__ void seq_arrive(unsigned* c) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
+}
+// Polls (bounded) until all ncta CTAs have arrived on counter c.
+__device__ __forceinline__ void seq_wait(const unsigned* c, int ncta, unsigned* status) {
+    uint32_t i = 0;
+    while (ld_acquire_gpu(c) < (unsigned)ncta) {
+        if (++i > kSpinTries) {
+            record_error(status, kDevTimeout);
+            break;
+        }
+    }
+}
+
 // The CTAs of one sequence meet here: each arrives on counter c, then polls
 // (bounded) until all ncta have; memory written before the meeting by the
 // group's threads of any of them is visible to all after it.  Called by a
@@ -164,16 +181,8 @@ template <int NT>
 __device__ void seq_barrier(unsigned* c, int ncta, unsigned* status, int bar, int lt) {
     gsync<NT>(bar);
     if (lt == 0) {
-        // release: the group's earlier writes (ordered before by the barrier)
-        // are visible to whoever acquires the count
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
-        uint32_t i = 0;
-        while (ld_acquire_gpu(c) < (unsigned)ncta) {
-            if (++i > kSpinTries) {
-                record_error(status, kDevTimeout);
-                break;
-            }
-        }
+        seq_arrive(c);
+        seq_wait(c, ncta, status);
     }
     gsync<NT>(bar);
 }
@@ -566,22 +575,48 @@ __global__ void __launch_bounds__(kThreads, 1)
     int def_full = 0;
     if (warp < 8) {
         if (!sel_all) {
-            // keys whose digit is above D1 are selected whatever tau is (thread t owns
-            // keys [t*ch, (t+1)*ch), so they stay in position order)
+            // keys whose digit is above D1 are selected whatever tau is: listed for
+            // the gather; keys of digit D1 are published as candidates for exchange 2
+            // (thread t owns keys [t*ch, (t+1)*ch), so both stay in position order;
+            // the two counts share one scan, 16 bits each)
             const int ch = (nk + kMainThreads - 1) / kMainThreads;
             const int c_lo = min(nk, tid * ch), c_hi = min(nk, c_lo + ch);
             int mine = 0;
-            for (int i = c_lo; i < c_hi; ++i) mine += (skeys[i] >> 20) > D1 ? 1 : 0;
+            for (int i = c_lo; i < c_hi; ++i) {
+                const uint32_t d = skeys[i] >> 20;
+                mine += d > D1 ? 1 : (d == D1 ? 1 << 16 : 0);
+            }
             int tot;
-            int at = grp_excl_scan<kMainThreads>(mine, tid, kConsBar, misc + 32, tot);
+            const int at0 = grp_excl_scan<kMainThreads>(mine, tid, kConsBar, misc + 32, tot);
+            const int tot_def = tot & 0xFFFF, tot_c = tot >> 16;
+            unsigned cbase = 0;
+            if (tid == 0 && tot_c) cbase = atomicAdd(sync + 4, (unsigned)tot_c);  // used after def_ready
+            int at = at0 & 0xFFFF;
             for (int i = c_lo; i < c_hi; ++i)
                 if ((skeys[i] >> 20) > D1) {
                     if (at < P.sel_cap) spos[at] = k0 + i;
                     ++at;
                 }
-            const int cnt_def = min(tot, P.sel_cap);
+            const int cnt_def = min(tot_def, P.sel_cap);
             def_full = cnt_def / kGK * kGK;
             if (tid == 0) ssel[4] = cnt_def;
+            gsync<kMainThreads>(kConsBar);
+            if (tid == 0) {
+                ptx::mbar_arrive(def_ready);  // the gather starts
+                misc[kMiscCBase] = (int)cbase;
+            }
+            gsync<kMainThreads>(kConsBar);
+            uint2* cand = P.cand + (int64_t)b * P.ns;
+            int ca = misc[kMiscCBase] + (at0 >> 16);
+            for (int i = c_lo; i < c_hi; ++i) {
+                const uint32_t key = skeys[i];
+                if ((key >> 20) == D1) {
+                    if (ca < P.ns) cand[ca] = make_uint2(key, (uint32_t)(k0 + i));
+                    ++ca;
+                }
+            }
+            gsync<kMainThreads>(kConsBar);
+            if (tid == 0) seq_arrive(sync + 1);  // exchange 2: this CTA's candidates are out
         } else {
             for (int i = tid; i < nk; i += kMainThreads) spos[i] = k0 + i;
             def_full = nk;
@@ -594,8 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (P.idx) P.gsel[(int64_t)b * P.ncta + j] = nk;
             }
         }
-        gsync<kMainThreads>(kConsBar);
-        if (tid == 0) ptx::mbar_arrive(def_ready);
+        if (sel_all) {
+            gsync<kMainThreads>(kConsBar);
+            if (tid == 0) ptx::mbar_arrive(def_ready);
+        }
     }
 
     // ======================================================== C: gather + attention
@@ -799,27 +836,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         need1 = misc[1];
         int* rmisc = misc + 48;  // find_bin results [0..2], tie counter [3], scan scratch [32..]
         uint2* cand = P.cand + (int64_t)b * P.ns;
-        // thread rt owns keys [rt*ch, (rt+1)*ch); one range of the candidate list
-        // is reserved for the whole CTA
+        // thread rt owns keys [rt*ch, (rt+1)*ch)
         const int ch = (nk + NT - 1) / NT;
         const int c_lo = min(nk, rt * ch), c_hi = min(nk, c_lo + ch);
-        {
-            int mine = 0;
-            for (int i = c_lo; i < c_hi; ++i) mine += (skeys[i] >> 20) == D1 ? 1 : 0;
-            int tot;
-            int at = grp_excl_scan<NT>(mine, rt, kRefBar, rmisc + 32, tot);
-            if (rt == 0) rmisc[4] = tot ? (int)atomicAdd(sync + 4, (unsigned)tot) : 0;
-            gsync<NT>(kRefBar);
-            at += rmisc[4];
-            for (int i = c_lo; i < c_hi; ++i) {
-                const uint32_t key = skeys[i];
-                if ((key >> 20) == D1) {
-                    if (at < P.ns) cand[at] = make_uint2(key, (uint32_t)(k0 + i));
-                    ++at;
-                }
-            }
-        }
-        seq_barrier<NT>(sync + 1, P.ncta, P.status, kRefBar, rt);
+        // exchange 2: every CTA's candidates are out (published by warps 0-7)
+        if (rt == 0) seq_wait(sync + 1, P.ncta, P.status);
+        gsync<NT>(kRefBar);
         {
             // no CTA reads the summed histogram any more: clear a share of it
             unsigned* gh = P.ghist + (int64_t)b * 4096;
@@ -827,12 +849,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lo = j * per, hi = min(4096, lo + per);
             for (int i = lo + rt; i < hi; i += NT) gh[i] = 0u;
         }
+        // the first 8 * NT list entries are loaded with the count (entries past it
+        // are discarded), the rest, if any, once the count is known
+        uint2 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = __ldcg(cand + min(rt + k * NT, P.ns - 1));
         const int C = min((int)__ldcg(sync + 4), P.ns);
         const bool in_smem = C <= kCandSmem;
         uint2* sc = reinterpret_cast<uint2*>(ring + kCandOff);
         if (in_smem) {
-            for (int i0 = 0; i0 < C; i0 += 8 * NT) {  // 8 loads in flight per thread
-                uint2 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = rt + k * NT;
+                if (i < C) sc[i] = v[k];
+            }
+            for (int i0 = 8 * NT; i0 < C; i0 += 8 * NT) {  // 8 loads in flight per thread
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int i = i0 + rt + k * NT;
