@@ -17,18 +17,21 @@
 //  B. The exact top-M threshold, agreed by the sequence's CTAs through global
 //     memory.  Exchange 1: the CTA histograms are summed and every CTA finds
 //     the 12-bit digit D1 holding the M-th largest key.  Keys above D1 are
-//     selected whatever the exact threshold is, so warps 0-7 list this CTA's
-//     at once and the gather starts.  Meanwhile warps 9-11 refine: exchange 2
-//     publishes the keys of digit D1 as (key, position) candidates, from which
-//     each CTA finds the exact M-th key tau by two 10-bit refinements and how
-//     many keys equal to tau are kept (the lowest positions); the CTA's
-//     selected keys of digit D1 are then appended to its list.
-//  C. The K and V rows of the listed positions (all KV heads of a position
-//     are one row) arrive by 1-D bulk copies in a ring of 16-key stages, filled
-//     by warp 8 and consumed by warps 0-7: tensor-core scores and P.V (keys on
-//     the MMA M side, the query heads of a GQA group on N) with an online
-//     softmax.  The partial (max, sum, output) of every query head goes to
-//     global memory.
+//     selected whatever the exact threshold is: warps 0-7 list this CTA's in
+//     one pass that also publishes its keys of digit D1 as (key, position)
+//     candidates and adds their bits [19:10] to the sequence's second-digit
+//     histogram (exchange 2), and the gather starts.  Meanwhile warps 9-11
+//     refine: the second digit from that histogram, the third from the
+//     candidates, giving the exact M-th key tau and how many keys equal to
+//     tau are kept (the lowest positions); the CTA's selected keys of digit D1
+//     are then appended to its list.
+//  C. The K rows of the listed positions (all KV heads of a position are one
+//     row) arrive by 1-D bulk copies of warp 8 in a ring of 16-key stages; each
+//     attention warp (0-7) fetches its own KV head's part of the V rows by
+//     16-byte cp.async copies and consumes the stages on the tensor cores
+//     (keys on the MMA M side, the query heads of a GQA group on N) with an
+//     online softmax.  The partial (max, sum, output) of every query head goes
+//     to global memory.
 //  D. After exchange 3: every CTA writes its share of the index row (when
 //     asked for), merges the partials of a few query heads, gates them with
 //     the linear branch and writes o; z advances in the elu+1 mode.
@@ -132,6 +135,7 @@ struct CoopParams {
     int32_t* count;
     unsigned* status;
     unsigned* ghist;    // [B][4096] sums of the CTA histograms (zero between calls)
+    unsigned* ghist2;   // [B][1024] histogram of bits [19:10] of the keys of digit D1 (zero between calls)
     unsigned* sync;     // [B][32]: arrivals of the 3 exchanges, departures, candidate count
     float* olin;        // [B][H_q][kD]
     float* part;        // [B][ncta][H_q][kD + 2]
@@ -607,12 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             gsync<kMainThreads>(kConsBar);
             uint2* cand = P.cand + (int64_t)b * P.ns;
+            unsigned* gh2 = P.ghist2 + (int64_t)b * 1024;
             int ca = misc[kMiscCBase] + (at0 >> 16);
             for (int i = c_lo; i < c_hi; ++i) {
                 const uint32_t key = skeys[i];
                 if ((key >> 20) == D1) {
                     if (ca < P.ns) cand[ca] = make_uint2(key, (uint32_t)(k0 + i));
                     ++ca;
+                    atomicAdd(gh2 + ((key >> 10) & 1023u), 1u);  // the sequence's second digit
                 }
             }
             gsync<kMainThreads>(kConsBar);
@@ -854,6 +860,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint2 v[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = __ldcg(cand + min(rt + k * NT, P.ns - 1));
+        // with them, the sequence's histogram of key bits [19:10] over digit D1
+        const uint4* gh2 = reinterpret_cast<const uint4*>(P.ghist2 + (int64_t)b * 1024);
+        constexpr int kH2 = (256 + NT - 1) / NT;
+        uint4 h2[kH2];
+#pragma unroll
+        for (int k = 0; k < kH2; ++k)
+            if (rt + k * NT < 256) h2[k] = __ldcg(gh2 + rt + k * NT);
         const int C = min((int)__ldcg(sync + 4), P.ns);
         const bool in_smem = C <= kCandSmem;
         uint2* sc = reinterpret_cast<uint2*>(ring + kCandOff);
@@ -877,10 +890,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         auto cand_at = [&](int i) { return in_smem ? sc[i] : __ldcg(cand + i); };
-        // second digit: key bits [19:10]
-        for (int i = rt; i < 1024; i += NT) shist[i] = 0u;
-        gsync<NT>(kRefBar);
-        for (int i = rt; i < C; i += NT) atomicAdd(shist + ((cand_at(i).x >> 10) & 1023u), 1u);
+        // second digit: key bits [19:10], from the histogram the CTAs built
+#pragma unroll
+        for (int k = 0; k < kH2; ++k)
+            if (rt + k * NT < 256) reinterpret_cast<uint4*>(shist)[rt + k * NT] = h2[k];
         gsync<NT>(kRefBar);
         find_bin<NT>(shist, 1024, need1, rmisc, rt, kRefBar);
         const uint32_t D2 = (uint32_t)rmisc[0];
@@ -1003,6 +1016,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = misc[4] + cnt + tid; i < P.M; i += kThreads) row[i] = -1;
     }
     if (j == 0 && tid == 0 && P.count) P.count[b] = min(P.M, n);
+    if (!sel_all) {
+        // every CTA read the second-digit histogram before exchange 3: clear a share
+        unsigned* gh2 = P.ghist2 + (int64_t)b * 1024;
+        const int per = (1024 + P.ncta - 1) / P.ncta;
+        const int lo = j * per, hi = min(1024, lo + per);
+        for (int i = lo + tid; i < hi; i += kThreads) gh2[i] = 0u;
+    }
     {
         constexpr int kChunk = 16;  // partials loaded together
         const int c = tid & (kD - 1), sub = tid / kD;
@@ -1163,6 +1183,7 @@ cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
     char* w8 = (char*)ws;
     P.status = (unsigned*)ws;
     P.ghist = (unsigned*)(w8 + decode_hist_offset());
+    P.ghist2 = (unsigned*)(w8 + decode_hist2_offset(s.B));
     P.sync = (unsigned*)(w8 + decode_sync_offset(s.B));
     P.olin = (float*)(w8 + pl.olin);
     P.part = (float*)(w8 + pl.part);

@@ -9,10 +9,11 @@ namespace lisa {
 
 // Decode-step workspaces start with state that is zero between calls, at
 // offsets that depend on B only, so that one workspace serves a batch at every
-// context length: [status | key histograms, B x 4096 u32 | barrier lines,
-// B x 128 bytes | scratch of the call].
+// context length: [status | key histograms, B x 4096 u32 | second-digit
+// histograms, B x 1024 u32 | barrier lines, B x 128 bytes | scratch of the call].
 inline size_t decode_hist_offset() { return kStatusBytes; }
-inline size_t decode_sync_offset(int B) { return kStatusBytes + (size_t)B * 4096 * 4; }
+inline size_t decode_hist2_offset(int B) { return kStatusBytes + (size_t)B * 4096 * 4; }
+inline size_t decode_sync_offset(int B) { return decode_hist2_offset(B) + (size_t)B * 1024 * 4; }
 inline size_t decode_scratch_offset(int B) { return decode_sync_offset(B) + (size_t)B * 128; }
 
 // Decode step: one cooperative kernel over all SMs (decode_coop.cu) when it
