@@ -121,6 +121,12 @@ def test_decode_1p5b_head_layout():
     run_decode_case(inputs.PREFILL_1P5B.with_(B=4, n=4096, M=512))
 
 
+def test_decode_one_kv_head():
+    """Eight query heads over a single KV head: 256-byte K/V rows, the deepest
+    stage ring and no V requests ahead of the current stage."""
+    run_decode_case(inputs.DECODE_7B.with_(B=3, n=5000, M=512, H_q=8, H_kv=1))
+
+
 def test_decode_fused_matches_generic_path_outputs_shape():
     """The fused path and a second identical call agree (the step is deterministic)."""
     wl = inputs.DECODE_7B.with_(B=2, n=3000, M=256)
