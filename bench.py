@@ -727,6 +727,10 @@ def oracle_decode_sample(wl, seqs: int, budget_s: float):
 
 
 def run_reference(args, wl):
+    # rank 0 is the only worker of this arm, so it takes every core it may run
+    # on (a multi-process launcher sets OMP_NUM_THREADS=1 for each rank)
+    from oracle import ref
+    ref.set_num_threads(len(os.sched_getaffinity(0)))
     tok_s, cores, note = oracle_decode_sample(wl, seqs=wl.B, budget_s=max(5.0, args.cpu_seconds))
     return {
         "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
