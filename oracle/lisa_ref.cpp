@@ -96,13 +96,15 @@ void ref_index_scores(const RefDims* D, const float* q_I, const float* k_I,
                       const float* w, int64_t w_tok_stride,
                       const int32_t* rows, int32_t R, double* scores) {
     const int L = D->n_past + D->T;
-#pragma omp parallel for collapse(2) schedule(dynamic)
+    // one (sequence, row, key) entry per iteration: a decode step (one row per
+    // sequence) still spreads over every host core
+#pragma omp parallel for collapse(3) schedule(dynamic, 256)
     for (int b = 0; b < D->B; ++b) {
         for (int r = 0; r < R; ++r) {
-            const int t = row_token(rows, r);
-            const int p = D->n_past + t;
-            double* out = scores + ((int64_t)b * R + r) * L;
             for (int s = 0; s < L; ++s) {
+                const int t = row_token(rows, r);
+                const int p = D->n_past + t;
+                double* out = scores + ((int64_t)b * R + r) * L;
                 if (s > p) { out[s] = -INFINITY; continue; }
                 double total = 0.0;
                 for (int j = 0; j < D->H_I; ++j) {
@@ -193,13 +195,14 @@ void ref_sparse_attn(const RefDims* D, const float* q, const float* k_cache,
                      const float* v_cache, const int32_t* rows, int32_t R,
                      const int32_t* idx, const int32_t* count, double* o) {
     const int group = D->H_q / D->H_kv;
-#pragma omp parallel for collapse(2) schedule(dynamic)
+    // one (sequence, row, query head) per iteration
+#pragma omp parallel for collapse(3) schedule(dynamic)
     for (int b = 0; b < D->B; ++b) {
         for (int r = 0; r < R; ++r) {
-            const int t = row_token(rows, r);
-            const int32_t* pos = idx + ((int64_t)b * R + r) * D->M;
-            const int npos = count[(int64_t)b * R + r];
             for (int h = 0; h < D->H_q; ++h) {
+                const int t = row_token(rows, r);
+                const int32_t* pos = idx + ((int64_t)b * R + r) * D->M;
+                const int npos = count[(int64_t)b * R + r];
                 const float* qh = q + (((int64_t)b * D->T + t) * D->H_q + h) * D->d;
                 double* out = o + (((int64_t)b * R + r) * D->H_q + h) * D->d;
                 attend(D, qh, k_cache, v_cache, b, h / group, pos, npos, out);
