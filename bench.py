@@ -52,16 +52,17 @@ def _peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def decode_bytes(wl) -> dict:
+def decode_bytes(wl, elu1: bool = False) -> dict:
     """Algorithmic HBM bytes of one decode step (per sequence and total).
 
     Keys are read once (k_I scan over the n cached positions), only the
-    min(M, n) selected K/V rows are gathered, the fp32 state is read and
-    written once, plus the step's small inputs and outputs."""
+    min(M, n) selected K/V rows are gathered, the fp32 state (and, with the
+    elu+1 feature map, its normaliser z) is read and written once, plus the
+    step's small inputs and outputs."""
     n, M = wl.n, wl.M
     scan = n * wl.H_Ik * wl.d_I * 2
     gather = min(M, n) * wl.H_kv * wl.d * 2 * 2
-    state = wl.H_kv * wl.d * wl.d * 4 * 2
+    state = wl.H_kv * wl.d * wl.d * 4 * 2 + (wl.H_kv * wl.d * 4 * 2 if elu1 else 0)
     small = (wl.H_q * wl.d * 2 * 2          # q, o
              + wl.H_q * wl.d * 2            # q_L (aliases q, counted once more for the LA read)
              + wl.H_kv * wl.d * 2 * 2 * 2   # k_new, v_new read + written to the cache
@@ -106,44 +107,61 @@ def _profiled_traffic(wl):
 
 
 class ClockSampler:
-    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    """nvidia-smi clock and throttle-reason samples, each stamped with the host
+    time it arrived, so that the samples inside the timed region can be told
+    from those around it."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_id: str):
+    def __init__(self, gpu_id: str, period_ms: int = 100):
         self.gpu = gpu_id
+        self.period_ms = period_ms
         self.proc = None
+        self.samples = []  # (host time, line)
+        self._reader = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.time(), ln))
 
     def __enter__(self):
+        import threading
+
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+            self._reader = threading.Thread(target=self._read, daemon=True)
+            self._reader.start()
         except Exception:
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             time.sleep(0.2)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self._reader is not None:
+                self._reader.join(timeout=5)
         return False
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock, maximum clock and throttle reasons of the samples
+        that arrived between host times t0 and t1 (all samples if not given)."""
         sm, smax, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
+        for ts, ln in self.samples:
+            if t0 is not None and not (t0 <= ts <= t1):
+                continue
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -156,9 +174,40 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "period_ms": self.period_ms, "window": "samples inside the timed region"}
+
+
+def time_blocks(step, steps: int, stream, min_seconds: float, max_blocks: int = 4000):
+    """Runs blocks of `steps` back-to-back steps with a CUDA event at every
+    block boundary (no host synchronisation in between) until about
+    `min_seconds` have passed on the device; returns the device time of each
+    block (ms) and the host times at which the timed region started and
+    ended.  The caller brackets it with a barrier and a synchronise."""
+    import torch
+
+    # size the run from one untimed block
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(stream)
+    for i in range(steps):
+        step(i)
+    b_.record(stream)
+    torch.cuda.synchronize()
+    est = max(a_.elapsed_time(b_), 1e-3)
+    blocks = int(min(max_blocks, max(1, math.ceil(min_seconds * 1e3 / est))))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(blocks + 1)]
+    torch.cuda.synchronize()
+    t0 = time.time()
+    ev[0].record(stream)
+    for k in range(blocks):
+        for i in range(steps):
+            step(k * steps + i)
+        ev[k + 1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    return [ev[k].elapsed_time(ev[k + 1]) for k in range(blocks)], t0, t1
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -245,7 +294,7 @@ def run_gpu(args, wl, rank, world, device):
         a = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"],
                              dv["w"], wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"],
                              kc, vc, kIc, S, None, o)
-        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S, kc=kc, vc=vc))
+        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S, kc=kc, vc=vc, kIc=kIc))
 
     def step(i):
         c = copies[i % len(copies)]
@@ -275,11 +324,12 @@ def run_gpu(args, wl, rank, world, device):
         for c in copies:
             assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
 
-    # the K timed steps run back to back between one pair of events on the
-    # launching stream (an event pair around every step would add its own gap
-    # to each step)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    # The K timed steps run back to back between CUDA events on the launching
+    # stream (an event pair around every step would add its own gap to each
+    # step).  Blocks of K steps repeat, with an event at each block boundary and
+    # no host synchronisation between them, until about --min-seconds of device
+    # time have passed, so that the clock samples taken inside the timed region
+    # are many; the reported time is the median block's.
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -288,16 +338,12 @@ def run_gpu(args, wl, rank, world, device):
     except Exception:
         gpu_id = str(device.index)
     with ClockSampler(gpu_id) as clk:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(i)
-        t_end.record(stream)
-        torch.cuda.synchronize()
+        blocks, w0, w1 = time_blocks(step, args.steps, stream, args.min_seconds)
     if world > 1:
         dist.barrier()
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), device, world)
+    total_ms = max_over_ranks(statistics.median(blocks), device, world)
 
     # ---- end to end through the public API with host buffers
     pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
@@ -360,11 +406,198 @@ def run_gpu(args, wl, rank, world, device):
                      "launch_us": avg_s * 1e6},
         "e2e": {"value": job_throughput(B, world, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": DECODE_KERNELS_PER_STEP * args.steps,
-        "clocks": clk.summary(),
+        "timing": {"blocks": len(blocks), "steps_per_block": args.steps,
+                   "block_ms_median": statistics.median(blocks), "block_ms_min": min(blocks),
+                   "block_ms_max": max(blocks), "timed_region_s": w1 - w0,
+                   "what": "blocks of K steps back to back, an event at each block boundary; "
+                           "value and ms_per_step from the median block (max over ranks)"},
+        "gpu_launches": DECODE_KERNELS_PER_STEP * args.steps * len(blocks),
+        "clocks": clk.summary(w0, w1),
     }
     line.update(extra)
     return line
+
+
+# ----------------------------------------------------------------------------- helpers
+def graph_timed(calls, steps: int, warmup: int):
+    """Captures one CUDA graph per call (each a closure issuing one library call
+    on the current stream) and replays them in rotation: `warmup` untimed
+    replays, then `steps` between one event pair on the launching stream.
+    Returns the device time per replay in ms."""
+    import torch
+
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    graphs = []
+    for c in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            c()
+        graphs.append(g)
+    cur = torch.cuda.current_stream()
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(cur)
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    b_.record(cur)
+    torch.cuda.synchronize()
+    ms = a_.elapsed_time(b_) / steps
+    del graphs
+    return ms
+
+
+def hbm_roof(nbytes: float, ms: float) -> dict:
+    hbm_peak, _, peak_kind = _peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "algorithmic_bytes_per_launch": nbytes, "achieved": gbs,
+            "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "peak_kind": peak_kind,
+            "traffic": None}
+
+
+def device_decode_state(wl, device, seed: int):
+    """Seeded synthetic decode state drawn on the device with torch's generator,
+    for the timing-only lines (drawing 32 sequences of 64K tokens through the
+    per-block host streams would take minutes).  Same recipe as the workload
+    generator: N(0, sigma^2) values, 1% of positions per sequence planted with
+    3 sigma sqrt(dim) along one shared unit direction in k and k_I, bf16."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    B, n = wl.B, wl.n
+
+    def rn(*shape, scale=wl.sigma):
+        return (torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * scale).to(bf)
+
+    kc = torch.empty(B, n, wl.H_kv, wl.d, dtype=bf, device=device)
+    vc = torch.empty_like(kc)
+    kI = torch.empty(B, n, wl.H_Ik, wl.d_I, dtype=bf, device=device)
+    u = torch.randn(wl.d, generator=g, device=device)
+    uI = torch.randn(wl.d_I, generator=g, device=device)
+    u, uI = u / u.norm(), uI / uI.norm()
+    cnt = n // 100
+    for b in range(B):  # one sequence at a time keeps the fp32 temporaries small
+        kc[b] = rn(n, wl.H_kv, wl.d)
+        vc[b] = rn(n, wl.H_kv, wl.d)
+        kI[b] = rn(n, wl.H_Ik, wl.d_I)
+        if cnt:
+            pos = torch.randperm(n, generator=g, device=device)[:cnt]
+            kc[b, pos] = (kc[b, pos].float() + 3 * wl.sigma * math.sqrt(wl.d) * u).to(bf)
+            kI[b, pos] = (kI[b, pos].float() + 3 * wl.sigma * math.sqrt(wl.d_I) * uI).to(bf)
+    p = n - 1
+    step = {"q": rn(B, 1, wl.H_q, wl.d), "q_I": rn(B, 1, wl.H_I, wl.d_I),
+            "w": torch.rand(B, 1, wl.H_I, generator=g, device=device),
+            "gate": rn(B, 1, wl.H_q, scale=1.0),
+            "k_new": kc[:, p:].clone(), "v_new": vc[:, p:].clone(), "k_I_new": kI[:, p:].clone()}
+    S = torch.randn(B, wl.H_kv, wl.d, wl.d, generator=g, device=device) * 0.05
+    return kc, vc, kI, S, step
+
+
+def coop_decode_kernel(B: int, n: int, window_M: int = 0, sms: int = 148) -> str:
+    """Which decode kernel the library's dispatch picks for B sequences at
+    context n: the cooperative kernel while each CTA's share of the positions
+    fits its shared memory (at most 8192), else the four-kernel form."""
+    m = min(window_M, n) if window_M else n
+    ncta = max(1, min(sms // max(1, B), (m + 15) // 16))
+    kpc = (-(-m // ncta) + 15) // 16 * 16
+    return ("k_decode_coop" if B <= sms and kpc <= 8192
+            else "k_decode_scan, k_decode_select, k_decode_attend, k_decode_combine")
+
+
+def run_sweep(args, device):
+    """The long-context decode sweep: B=32 sequences at every context of 4K-64K
+    with both budgets (tok/s and HBM fraction per point), the Stage-1 window
+    step at the same budgets (the sparse branch alone, no indexer scan: its
+    cost must stay flat in the context), and dense causal attention over the
+    same caches (the O(n) reference line)."""
+    import torch
+
+    from hybrid_linear_top_lightning_b200 import inputs, lisa
+
+    points, dense, window = [], [], {}
+    for n in inputs.SWEEP_CTX:
+        wl0 = inputs.sweep_workload(n, min(inputs.SWEEP_M))
+        kc0, vc0, kI0, S0, st0 = device_decode_state(wl0, device, seed=1000 + n)
+        ncopy = int(min(4, max(1, math.ceil(400e6 / decode_bytes(wl0)["total"]))))
+        copies = []
+        for r in range(ncopy):
+            if r == 0:
+                c = dict(kc=kc0, vc=vc0, kI=kI0, S=S0, st=st0)
+            else:
+                c = dict(kc=kc0.clone(), vc=vc0.clone(), kI=kI0.clone(), S=S0.clone(),
+                         st={k: v.clone() for k, v in st0.items()})
+            c["o"] = torch.empty(wl0.B, 1, wl0.H_q, wl0.d, dtype=torch.bfloat16, device=device)
+            copies.append(c)
+        for M in inputs.SWEEP_M:
+            wl = inputs.sweep_workload(n, M)
+            D = lisa.make_dims(wl.B, 1, n - 1, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, M)
+            calls_d, calls_w = [], []
+            for c in copies:
+                st = c["st"]
+                a = lisa.decode_args(st["q"], st["k_new"], st["v_new"], st["q_I"], st["k_I_new"],
+                                     st["w"], wl.H_I, st["q"], st["k_new"], st["v_new"],
+                                     st["gate"], c["kc"], c["vc"], c["kI"], c["S"], None, c["o"])
+                ws = lisa.workspace(D, lisa.LISA_OP_DECODE_STEP, device)
+                calls_d.append(lambda a=a, ws=ws: lisa.lisa_decode_step(D, a, ws))
+                calls_w.append(lambda a=a, ws=ws: lisa.lisa_decode_step_window(D, a, ws))
+                c.setdefault("ws", []).append(ws)
+            ms_d = graph_timed(calls_d, args.steps, args.warmup)
+            ms_w = graph_timed(calls_w, args.steps, args.warmup)
+            for c in copies:
+                for ws in c.pop("ws"):
+                    assert lisa.lisa_check_status(ws) == lisa.LISA_OK
+            db, wb = decode_bytes(wl), window_bytes(wl)
+            points.append({"context": n, "M": M, "B": wl.B, "us_per_step": ms_d * 1e3,
+                           "value": wl.B / (ms_d / 1e3), "unit": "tok/s",
+                           "kernel": coop_decode_kernel(wl.B, n),
+                           "l2": f"{ncopy} state copies in rotation",
+                           "roofline": hbm_roof(db["total"], ms_d)})
+            window.setdefault(M, []).append({"context": n, "us_per_step": ms_w * 1e3,
+                                             "kernel": coop_decode_kernel(wl.B, n, M),
+                                             "roofline": hbm_roof(wb["total"], ms_w)})
+        # dense causal attention over the same caches (one query token per sequence)
+        Dd = lisa.make_dims(wl0.B, 1, n - 1, n, wl0.H_q, wl0.H_kv, wl0.d, wl0.H_I, wl0.H_Ik,
+                            wl0.d_I, wl0.M)
+        calls, wss = [], []
+        for c in copies:
+            ws = lisa.workspace(Dd, lisa.LISA_OP_DENSE_ATTN, device)
+            wss.append(ws)
+            calls.append(lambda c=c, ws=ws: lisa.lisa_dense_attn(Dd, c["st"]["q"], c["kc"],
+                                                                c["vc"], c["o"], ws))
+        ms = graph_timed(calls, max(4, args.steps // 4), args.warmup)
+        for ws in wss:
+            assert lisa.lisa_check_status(ws) == lisa.LISA_OK
+        nbytes = wl0.B * (n * wl0.H_kv * wl0.d * 2 * 2 + 2 * wl0.H_q * wl0.d * 2)
+        dense.append({"context": n, "B": wl0.B, "us_per_call": ms * 1e3,
+                      "value": wl0.B / (ms / 1e3), "unit": "tok/s",
+                      "roofline": hbm_roof(nbytes, ms)})
+        del copies, kc0, vc0, kI0, S0, st0
+        torch.cuda.empty_cache()
+    # the O(M)-not-O(n) check: at a fixed budget the sparse branch's time stays
+    # flat across the contexts (window step), while the full step grows with
+    # the indexer scan (128 bytes per cached token per sequence)
+    flat = {}
+    for M, rows in window.items():
+        us = [r["us_per_step"] for r in rows]
+        full = [p["us_per_step"] for p in points if p["M"] == M]
+        flat[str(M)] = {"contexts": [r["context"] for r in rows], "window_us": us,
+                        "window_max_over_min": max(us) / min(us), "decode_us": full,
+                        "decode_max_over_min": max(full) / min(full),
+                        "scan_bytes_per_seq": [128 * r["context"] for r in rows],
+                        "gather_bytes_per_seq": [min(int(M), r["context"]) * 2048 for r in rows]}
+    return {"what": "decode step at B=32 over every (context, budget) point, with the "
+                    "Stage-1 window step at the same budgets and dense causal attention "
+                    "(lisa_dense_attn) on the same caches",
+            "data": "seeded synthetic caches drawn on the device (torch generator; the "
+                    "workload recipe: N(0, 1/128), 1% planted heavy keys, bf16)",
+            "points": points, "dense": dense,
+            "window": {str(M): rows for M, rows in window.items()},
+            "o_of_m_check": flat}
 
 
 # ----------------------------------------------------------------------------- next rows
@@ -420,6 +653,28 @@ def run_next_rows(args, wl, copies, D, stream):
                      "achieved": wb["total"] / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": wb["total"] / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
                      "traffic": None}}
+    # ---- the elu+1 feature map with its normaliser z (the same state copies,
+    # a positive z each); the step also advances z
+    De = lisa.make_dims(wl.B, 1, wl.n - 1, wl.n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik,
+                        wl.d_I, wl.M, phi=lisa.LISA_PHI_ELU1_NORM)
+    calls = []
+    for c in copies:
+        dv = c["dv"]
+        z = torch.rand(wl.B, wl.H_kv, wl.d, device=stream.device) * 20.0 + 1.0
+        ae = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"],
+                              dv["w"], wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"],
+                              c["kc"], c["vc"], c["kIc"], c["S"], z, c["o"])
+        calls.append(lambda ae=ae, ws=c["ws"]: lisa.lisa_decode_step(De, ae, ws))
+    ms = graph_timed(calls, args.steps, args.warmup)
+    for c in copies:
+        assert lisa.lisa_check_status(c["ws"], cur) == lisa.LISA_OK
+    eb = decode_bytes(wl, elu1=True)
+    out["elu1"] = {
+        "what": "decode step with the elu+1 feature map and its normaliser "
+                "(phi = LISA_PHI_ELU1_NORM), one cooperative kernel",
+        "value": wl.B / (ms / 1e3), "unit": "tok/s", "us_per_step": ms * 1e3,
+        "roofline": hbm_roof(eb["total"], ms)}
+
     # ---- the paper's indexer form: a key per indexer head (H_Ik = H_I = 8), w = 1
     from hybrid_linear_top_lightning_b200 import inputs
 
@@ -640,6 +895,9 @@ def run_prefill(args, wl, device):
     o_sp, o_lin = torch.empty_like(o), torch.empty_like(o)
     idx = torch.empty(B, n, wl.M, dtype=torch.int32, device=device)
     cnt = torch.empty(B, n, dtype=torch.int32, device=device)
+    De = lisa.make_dims(B, n, 0, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                        chunk=wl.chunk, phi=lisa.LISA_PHI_ELU1_NORM)
+    z = torch.zeros(B, wl.H_kv, wl.d, device=device)
     ws = lisa.workspace(D, lisa.LISA_OP_PREFILL, device)
     args_p = lisa.prefill_args(q, k, v, qI, kI, w, wl.H_I, q, k, v, gl, S, None, o, idx, cnt)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
@@ -650,6 +908,7 @@ def run_prefill(args, wl, device):
         "topm": lambda: lisa.lisa_topm(D, qI, kI, w, wl.H_I, idx, cnt, ws, stream),
         "sparse_attn": lambda: lisa.lisa_sparse_attn(D, q, k, v, idx, cnt, o_sp, ws, stream),
         "linear": lambda: lisa.lisa_linear_prefill(D, q, k, v, S, None, o_lin, ws, stream),
+        "linear_elu1": lambda: lisa.lisa_linear_prefill(De, q, k, v, S, z, o_lin, ws, stream),
         "gate": lambda: lisa.lisa_gate_fuse(D, gl, o_lin, o_sp, o, stream),
     }
     steps = max(1, args.prefill_steps)
@@ -674,10 +933,13 @@ def run_prefill(args, wl, device):
     whole_s = times["whole"] / 1e3
     idx_tf = work["indexer"] / (times["topm"] / 1e3) / 1e12
     lin_tf = work["linear"] / (times["linear"] / 1e3) / 1e12
+    lin_e_tf = work["linear"] / (times["linear_elu1"] / 1e3) / 1e12
     return {
         "workload": wl.name, "B": B, "n": n, "M": wl.M, "H_q": wl.H_q, "H_kv": wl.H_kv,
         "value": B * n / whole_s, "unit": "tok/s", "ms": times["whole"], "steps": steps,
         "stage_ms": {k_: v_ for k_, v_ in times.items() if k_ != "whole"},
+        "stage_note": "linear_elu1 is the linear branch with the elu+1 feature map and its "
+                      "normaliser (not part of the whole-module time, which uses the identity)",
         "gpu_launches_per_prefill": 7,
         "l2": "256 MB buffer written before every timed call",
         "work": {"indexer_gflop": work["indexer"] / 1e9, "sparse_gflop": work["sparse"] / 1e9,
@@ -688,42 +950,57 @@ def run_prefill(args, wl, device):
             "frac": work["total"] / whole_s / 1e12 / tc_burst,
             "indexer_tflops_incl_select": idx_tf, "indexer_frac_incl_select": idx_tf / tc_burst,
             "linear_tflops": lin_tf, "linear_frac": lin_tf / tc_burst,
+            "linear_elu1_tflops": lin_e_tf, "linear_elu1_frac": lin_e_tf / tc_burst,
             "sparse_gather_gbs": work["gather_bytes"] / (times["sparse_attn"] / 1e3) / 1e9,
             "traffic": None},
     }
 
 
 # ----------------------------------------------------------------------------- CPU oracle
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs(wl, seqs: int):
+    """The seeded inputs of `seqs` sequences of the decode workload (drawn once)."""
+    from hybrid_linear_top_lightning_b200 import inputs
+
+    key = (wl.name, seqs)
+    if key not in _ORACLE_INPUTS:
+        gen = inputs.Generator(wl.with_(B=seqs))
+        n, p = wl.n, wl.n - 1
+        x = {k: gen.batch(k, 0, n) for k in ("k", "v", "k_I")}
+        x.update({k: gen.batch(k, p, n) for k in ("q", "q_I", "w", "gate")})
+        rng = np.random.default_rng(0)
+        x["S0"] = rng.standard_normal((seqs, wl.H_kv, wl.d, wl.d)) * 0.1
+        _ORACLE_INPUTS[key] = x
+    return _ORACLE_INPUTS[key]
+
+
 def oracle_decode_sample(wl, seqs: int, budget_s: float):
     """Time the oracle's decode step on `seqs` sequences of the workload, repeated
     until about `budget_s` seconds have passed.  Returns (tok/s, threads, note)."""
-    from hybrid_linear_top_lightning_b200 import inputs
     from oracle import ref
 
-    gen = inputs.Generator(wl.with_(B=seqs))
+    x = _oracle_inputs(wl, seqs)
     n, p = wl.n, wl.n - 1
-    kc = gen.batch("k", 0, n)
-    vc = gen.batch("v", 0, n)
-    kI = gen.batch("k_I", 0, n)
-    q = gen.batch("q", p, n)
-    qI = gen.batch("q_I", p, n)
-    w = gen.batch("w", p, n)
-    gl = gen.batch("gate", p, n)
-    rng = np.random.default_rng(0)
-    S0 = rng.standard_normal((seqs, wl.H_kv, wl.d, wl.d)) * 0.1
     D = ref.Dims(B=seqs, T=1, n_past=p, N_max=n, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d, H_I=wl.H_I,
                  H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
+    kc, vc = x["k"], x["v"]
     reps = 0
     t0 = time.perf_counter()
     while True:
-        ref.forward(D, q, kc, vc, qI, kI, w, wl.H_I, q, kc[:, p:], vc[:, p:], gl, S0=S0)
+        ref.forward(D, x["q"], kc, vc, x["q_I"], x["k_I"], x["w"], wl.H_I, x["q"], kc[:, p:],
+                    vc[:, p:], x["gate"], S0=x["S0"])
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
     tok_s = reps * seqs / el
-    return tok_s, ref.num_threads(), (f"{reps} oracle decode steps of {seqs} sequences at "
-                                      f"context {n} (full step per sequence) in {el:.1f} s")
+    thr = ref.num_threads()
+    return tok_s, thr, (f"{reps} oracle decode steps of {seqs} sequences at context {n} "
+                        f"(the full step per sequence: indexer over every key, full sort, "
+                        f"sparse attention, linear branch, gate) in {el:.1f} s on {thr} "
+                        f"thread(s)")
 
 
 def run_reference(args, wl):
@@ -751,6 +1028,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="lisa", choices=["lisa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--min-seconds", type=float, default=1.5,
+                    help="device time of the timed region: blocks of --steps steps repeat "
+                         "until it has passed (clock samples inside it)")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false",
+                    help="skip the long-context sweep (B=32, contexts 4K-64K, both budgets, "
+                         "window and dense lines)")
     ap.add_argument("--rotate", type=int, default=4,
                     help="copies of the decode state used in rotation (inputs larger than L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -812,10 +1095,21 @@ def main():
             line["gate_channel"] = run_gate_channel(args, device)
         if args.prefill_steps > 0:
             line["prefill"] = run_prefill(args, wl_p, device)
+        if args.sweep:
+            line["sweep"] = run_sweep(args, device)
+            line["prefill_1p5b"] = run_prefill(args, inputs.PREFILL_1P5B, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            tok_s, cores, note = oracle_decode_sample(wl, seqs=2, budget_s=args.cpu_seconds)
+            from oracle import ref
+            ref.set_num_threads(len(os.sched_getaffinity(0)))
+            tok_s, cores, note = oracle_decode_sample(wl, seqs=wl.B, budget_s=args.cpu_seconds)
+            ref.set_num_threads(1)
+            tok_1, _, note_1 = oracle_decode_sample(wl, seqs=wl.B,
+                                                    budget_s=max(2.0, args.cpu_seconds / 2))
+            ref.set_num_threads(cores)
             line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores,
-                                    "kind": "oracle", "sample": note}
+                                    "kind": "oracle", "sample": note,
+                                    "single_thread": {"value": tok_1, "unit": UNIT, "cores": 1,
+                                                      "sample": note_1}}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

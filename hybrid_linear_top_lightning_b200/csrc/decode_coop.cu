@@ -166,11 +166,12 @@ __device__ __forceinline__ void gsync(int bar) {
 __device__ __forceinline__ void seq_arrive(unsigned* c) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(c) : "memory");
 }
-// Polls (bounded) until all ncta CTAs have arrived on counter c.
-__device__ __forceinline__ void seq_wait(const unsigned* c, int ncta, unsigned* status) {
+// Polls (at most `tries` times) until all ncta CTAs have arrived on counter c.
+__device__ __forceinline__ void seq_wait(const unsigned* c, int ncta, unsigned* status,
+                                         uint32_t tries = kSpinTries) {
     uint32_t i = 0;
     while (ld_acquire_gpu(c) < (unsigned)ncta) {
-        if (++i > kSpinTries) {
+        if (++i > tries) {
             record_error(status, kDevTimeout);
             break;
         }
@@ -180,13 +181,15 @@ __device__ __forceinline__ void seq_wait(const unsigned* c, int ncta, unsigned* 
 // The CTAs of one sequence meet here: each arrives on counter c, then polls
 // (bounded) until all ncta have; memory written before the meeting by the
 // group's threads of any of them is visible to all after it.  Called by a
-// group of NT threads (lt = thread index within the group).
+// group of NT threads (lt = thread index within the group).  `skip_arrival`
+// and `tries` serve the fault-injection hook of the workspace header only.
 template <int NT>
-__device__ void seq_barrier(unsigned* c, int ncta, unsigned* status, int bar, int lt) {
+__device__ void seq_barrier(unsigned* c, int ncta, unsigned* status, int bar, int lt,
+                            bool skip_arrival = false, uint32_t tries = kSpinTries) {
     gsync<NT>(bar);
     if (lt == 0) {
-        seq_arrive(c);
-        seq_wait(c, ncta, status);
+        if (!skip_arrival) seq_arrive(c);
+        seq_wait(c, ncta, status, tries);
     }
     gsync<NT>(bar);
 }
@@ -382,6 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nk = max(0, k1 - k0);
     const bool sel_all = P.window || n <= P.M;  // every position is kept: no scores needed
     unsigned* sync = P.sync + (int64_t)b * 32;
+    // Fault-injection hook (words 2-3 of the workspace header, zero in normal
+    // use): word 2 = 1 + the index of a CTA of every sequence that leaves out
+    // its arrival at exchange 1, word 3 = the poll limit of that exchange (0:
+    // the default).  Tests use it to watch a bounded wait give up.
+    uint2 hook = make_uint2(0u, 0u);
+    if (tid == 0) hook = __ldcg(reinterpret_cast<const uint2*>(P.status + 2));
 
     for (int i = tid; i < 4096; i += kThreads) shist[i] = 0u;
     if (tid == 0) {
@@ -536,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const unsigned c = shist[i];
             if (c) atomicAdd(gh + i, c);
         }
-        seq_barrier<kMainThreads>(sync + 0, P.ncta, P.status, kConsBar, tid);
+        seq_barrier<kMainThreads>(sync + 0, P.ncta, P.status, kConsBar, tid,
+                                  hook.x == (unsigned)j + 1u, hook.y ? hook.y : kSpinTries);
         // the summed histogram from L2: thread t holds bins [16t, 16t + 16)
         static_assert(4096 == 16 * kMainThreads, "16 bins per thread");
         unsigned hv[16];
@@ -1089,13 +1099,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
+// SM count of the current device (cached per device).
 int coop_num_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    constexpr int kMaxDev = 64;
+    static int sms_of[kMaxDev] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    int sms = (dev >= 0 && dev < kMaxDev) ? sms_of[dev] : 0;
+    if (sms <= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms <= 0)
             sms = 148;
+        if (dev >= 0 && dev < kMaxDev) sms_of[dev] = sms;
     }
     return sms;
 }

@@ -653,7 +653,13 @@ bool fast_decode_supported(const Shape& s, const lisa_decode_args& a, bool windo
 
 cudaError_t fast_decode_step(const Shape& s, const lisa_decode_args& a, void* ws, cudaStream_t st,
                              bool window) {
-    if (coop_decode_supported(s, a, window)) return coop_decode_step(s, a, ws, st, window);
+    if (coop_decode_supported(s, a, window)) {
+        const cudaError_t e = coop_decode_step(s, a, ws, st, window);
+        // a cooperative grid that does not fit the device right now takes the
+        // four-kernel form below
+        if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+        (void)cudaGetLastError();
+    }
     const Plan pl = make_plan(s);
     Params P;
     P.B = s.B; P.n = s.L; P.ns = pl.ns; P.N_max = s.N_max; P.H_q = s.H_q; P.H_kv = s.H_kv;

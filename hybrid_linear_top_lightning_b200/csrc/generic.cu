@@ -56,7 +56,7 @@ __global__ void k_index_scores(Shape s, const T* __restrict__ q_I, const T* __re
     extern __shared__ float sm[];
     float* qs = sm;                      // [H_I * d_I]
     float* ws = sm + s.H_I * s.d_I;      // [H_I]
-    const int row = blockIdx.y;
+    const int row = blockIdx.x;  // rows on x: B*T may exceed the 65535 limit of y
     const int b = row / s.T, t = row % s.T;
     const int p = s.n_past + t;
     const T* qrow = q_I + (int64_t)row * s.H_I * s.d_I;
@@ -65,7 +65,7 @@ __global__ void k_index_scores(Shape s, const T* __restrict__ q_I, const T* __re
     for (int j = threadIdx.x; j < s.H_I; j += blockDim.x)
         ws[j] = w[b * wb + (int64_t)t * w_tok_stride + j];
     __syncthreads();
-    const int key = blockIdx.x * blockDim.x + threadIdx.x;
+    const int key = blockIdx.y * blockDim.x + threadIdx.x;
     if (key >= s.L) return;
     float total = -INFINITY;
     if (key <= p) {
@@ -352,7 +352,8 @@ cudaError_t generic_index_scores(const Shape& s, const void* q_I, const void* k_
                                  int64_t w_tok_stride, float* scores, cudaStream_t st) {
     const int rows = s.B * s.T;
     if (rows == 0 || s.L == 0) return cudaSuccess;
-    dim3 grid((s.L + 127) / 128, rows);
+    if ((s.L + 127) / 128 > 65535) return cudaErrorInvalidValue;  // key blocks on y
+    dim3 grid(rows, (s.L + 127) / 128);
     const size_t smem = sizeof(float) * (s.H_I * s.d_I + s.H_I);
     if (s.dtype == LISA_BF16)
         k_index_scores<__nv_bfloat16><<<grid, 128, smem, st>>>(

@@ -20,7 +20,11 @@
 //    several host threads) race on it and must be serialised by the caller;
 //  - the first call on each device looks up the array's device address (a
 //    one-time set-up with that device current); make that first call before
-//    any stream capture begins.
+//    any stream capture begins.  The address belongs to the device's current
+//    context: after cudaDeviceReset the next call sees a new context and looks
+//    the address up again (that call, too, must come before any capture).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "lisa_internal.cuh"
@@ -35,18 +39,50 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Process-unique id of the current context (0 when the driver cannot say):
+// a reset device gets a new context, and with it a new id.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    }
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 // Device address of the scratch array on the current device (nullptr on
 // failure).  In host code the array's name is only a host-side stand-in, so the
-// address must come from cudaGetSymbolAddress with the device current.
+// address must come from cudaGetSymbolAddress with the device current; it is
+// looked up once per device and context.
 void* scratch_for_current_device() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_addr[dev] || ctx != g_scratch_ctx[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     return g_scratch_addr[dev];
 }

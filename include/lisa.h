@@ -45,14 +45,20 @@
  *    start of the workspace and returned by lisa_check_status.  The library
  *    never aborts, traps or prints.
  *  - Workspace: entry points that take `ws` need at least lisa_workspace_size()
- *    bytes of device memory, 256-byte aligned, ZERO-FILLED ONCE when allocated;
- *    the library keeps the first 256 bytes (status word) and re-initialises the
- *    rest itself.  A workspace must not be shared by calls that may run
- *    concurrently.  The decode steps keep state between calls in the workspace
- *    (key histograms and exchange counters, all zero again when a call ends) at
- *    offsets that depend on B only: one workspace, sized for the largest
- *    context, serves a batch as its context grows; zero-fill it again after B
- *    changes or after lisa_check_status has returned LISA_ERR_TIMEOUT.
+ *    bytes of device memory, 256-byte aligned, ZERO-FILLED when allocated.  The
+ *    first 256 bytes are a header: 32-bit word 0 is the status word, words 2-3
+ *    a fault-injection hook for tests (keep them zero: a non-zero word 2 makes
+ *    the decode step leave out one exchange arrival on purpose), the rest is
+ *    reserved.  A workspace must not be shared by calls that may run
+ *    concurrently.  Every entry point other than the decode steps uses the rest
+ *    as scratch that it initialises itself.  The decode steps
+ *    (lisa_decode_step, lisa_decode_step_window) instead keep state between
+ *    calls in their workspace (key histograms and exchange counters, all zero
+ *    again when a call ends) at offsets that depend on B only: one workspace,
+ *    sized for the largest context, serves a batch as its context grows.
+ *    Zero-fill a workspace again before a decode step uses it when another
+ *    entry point has used it since, when B has changed, or when
+ *    lisa_check_status has returned LISA_ERR_TIMEOUT.
  */
 #ifndef LISA_H_
 #define LISA_H_

@@ -117,6 +117,11 @@ def test_decode_elu1_feature_map():
     run_decode_case(inputs.DECODE_7B.with_(B=2, n=4000, M=512), phi=lisa.LISA_PHI_ELU1_NORM)
 
 
+def test_decode_7b_headline_elu1_full_size():
+    """The headline shape with the elu+1 feature map and its normaliser."""
+    run_decode_case(inputs.DECODE_7B, phi=lisa.LISA_PHI_ELU1_NORM)
+
+
 def test_decode_1p5b_head_layout():
     run_decode_case(inputs.PREFILL_1P5B.with_(B=4, n=4096, M=512))
 

@@ -1,6 +1,8 @@
 """GPU parity at the long-context decode sweep sizes (bf16): B=32 sequences,
-contexts 4096 .. 65536, budgets M in {512, 2048}, through lisa_decode_step,
-and the dense causal attention line (lisa_dense_attn) on the same caches.
+every context of 4096 .. 65536 with both budgets M in {512, 2048}, through
+lisa_decode_step (the cooperative kernel up to 32768, the four-kernel form at
+65536), and the dense causal attention line (lisa_dense_attn) on the same
+caches at every context.
 
 The whole batch runs on the GPU; the oracle checks sampled sequences (batch
 elements are independent).  The linear state is a seeded random input (the
@@ -84,11 +86,9 @@ def _sweep_case(n, M, dense):
         assert err_d <= TOL["bf16"], err_d
 
 
-@pytest.mark.parametrize("n,M", [(4096, 512), (4096, 2048), (16384, 512), (32768, 2048)])
+@pytest.mark.parametrize("M", inputs.SWEEP_M)
+@pytest.mark.parametrize("n", inputs.SWEEP_CTX)
 def test_decode_sweep_point(n, M):
-    _sweep_case(n, M, dense=False)
-
-
-@pytest.mark.parametrize("M", [512, 2048])
-def test_decode_sweep_64k_with_dense_line(M):
-    _sweep_case(65536, M, dense=(M == 2048))
+    """Every (context, budget) point of the sweep; the dense line (which does
+    not depend on M) is checked once per context, with the larger budget."""
+    _sweep_case(n, M, dense=(M == max(inputs.SWEEP_M)))

@@ -6,7 +6,7 @@ tensors).  This entry point keeps its scratch in a device array built into the
 library.  The test calls it through the C ABI twice in a row (the shared
 array keeps the previous call's contents) and checks that each result equals
 what lisa_topm, which takes a caller-provided workspace, returns for the same
-inputs.  It lives in its own file, collected last.
+inputs, and the oracle's selection.  It lives in its own file, collected last.
 """
 import numpy as np
 import pytest
@@ -62,6 +62,34 @@ def test_noalloc_topm_matches_workspace_topm_twice():
         np.testing.assert_array_equal(b_cnt, a_cnt)
         for bb in range(wl.B):
             check_topm(b_idx[bb], b_cnt[bb], a_idx[bb], a_cnt[bb], sc[bb])
+        # and both against the oracle's own selection (a full sort of its scores)
+        r_idx, r_cnt = ref.topm(Dr, sc)
+        for bb in range(wl.B):
+            check_topm(b_idx[bb], b_cnt[bb], r_idx[bb], r_cnt[bb], sc[bb])
+
+
+def test_noalloc_topm_more_rows_than_a_grid_column():
+    """70000 single-token sequences over 14 cached keys: more query rows than
+    the 65535 a launch grid's y dimension allows, within the 4 MiB array."""
+    wl = inputs.TINY.with_(B=70000, M=4)
+    T, n_past = 1, 13
+    L = n_past + T
+    # one seeded draw for the whole batch (the per-sequence streams of the
+    # workload generator would take minutes for 70000 sequences)
+    rng = np.random.default_rng(7)
+    q_I = torch.from_numpy(rng.standard_normal((wl.B, T, wl.H_I, wl.d_I), dtype=np.float32)).cuda()
+    k_I = torch.from_numpy(rng.standard_normal((wl.B, L, wl.H_Ik, wl.d_I), dtype=np.float32)).cuda()
+    w = torch.from_numpy(rng.random((wl.B, T, wl.H_I), dtype=np.float32)).cuda()
+    D = lisa.make_dims(wl.B, T, n_past, L, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M,
+                       dtype="f32")
+    a_idx, a_cnt, b_idx, b_cnt = _topm_both(D, q_I, k_I, w, wl.H_I)
+    Dr = ref.Dims(B=wl.B, T=T, n_past=n_past, N_max=L, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d,
+                  H_I=wl.H_I, H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
+    sc = ref.index_scores(Dr, q_I.cpu().numpy(), k_I.cpu().numpy(), w.cpu().numpy(), wl.H_I)
+    r_idx, r_cnt = ref.topm(Dr, sc)
+    for got_idx, got_cnt in ((a_idx, a_cnt), (b_idx, b_cnt)):
+        check_topm(got_idx.reshape(-1, wl.M), got_cnt.reshape(-1), r_idx.reshape(-1, wl.M),
+                   r_cnt.reshape(-1), sc.reshape(-1, L))
 
 
 def test_noalloc_rejects_calls_beyond_its_scratch():
