@@ -93,13 +93,15 @@ struct AttSrc {
 };
 
 // The position this thread copies in stage st of the list pos[0..cnt) (the
-// stage's first entry pads a short last stage; those keys are masked).
+// stage's first entry pads a short last stage; those keys are masked).  With
+// pos == nullptr the list is the run of positions iota0, iota0 + 1, ...
 template <int HKV>
-__device__ __forceinline__ int attn_stage_pos(const int* pos, int cnt, int st) {
+__device__ __forceinline__ int attn_stage_pos(const int* pos, int cnt, int st, int iota0 = 0) {
     using A = AttGeo<HKV>;
     if (st * A::keys >= cnt) return 0;
     const int jj = st * A::keys + threadIdx.x / A::tpk;
-    return pos[jj < cnt ? jj : st * A::keys];
+    const int e = jj < cnt ? jj : st * A::keys;
+    return pos ? pos[e] : iota0 + e;
 }
 
 // Issues this thread's 16-byte asynchronous copies of stage st into ring slot
@@ -216,15 +218,16 @@ __device__ __forceinline__ void attn_stage16(const uint32_t (&qf)[8][2], uint32_
 }
 
 // q: the row's query fragments (attn_load_q), `group` <= 8 heads per KV
-// head.  pos[0..cnt): positions (shared or global memory), gathered from
-// `src`; positions outside [0, src.p_max] are masked out and reported through
+// head.  pos[0..cnt): positions (shared or global memory; nullptr: the run
+// iota0 .. iota0 + cnt - 1), gathered from `src`; positions outside [0, src.p_max] are masked out and reported through
 // `status`.  `ring` holds AttGeo<HKV>::ring_bytes bytes, `spos` (shared
 // memory) kAttStages * AttGeo<HKV>::keys ints; both are clobbered.  The
 // result is valid in the warps with part == 0 (warp % wph == 0).
 template <int HKV, bool SPLIT = false>
 __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spos, const int* pos,
                                           int cnt, const AttSrc& src, float scale_log2,
-                                          unsigned* status, AttOut& out, uint64_t* kbar = nullptr) {
+                                          unsigned* status, AttOut& out, uint64_t* kbar = nullptr,
+                                          int iota0 = 0) {
     using A = AttGeo<HKV>;
     constexpr int GK = A::keys;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -233,7 +236,7 @@ __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spo
     const int key0 = part * 16;  // this warp's keys within a stage
     const int nst = (cnt + GK - 1) / GK;
     const int p_max = src.p_max;
-    auto load_pos = [&](int st) { return attn_stage_pos<HKV>(pos, cnt, st); };
+    auto load_pos = [&](int st) { return attn_stage_pos<HKV>(pos, cnt, st, iota0); };
     auto issue_stage = [&](int st, int raw) {
         attn_issue_stage<HKV, SPLIT>(ring, spos, cnt, st, raw, src, kbar);
     };

@@ -44,6 +44,16 @@ cudaError_t fast_attention(const Shape& s, const void* q, const void* k, const v
                            const int32_t* idx, const int32_t* count, void* o, void* ws,
                            cudaStream_t st);
 
+// Sparse attention of many query rows through a bit mask of the selections and
+// tcgen05 tiles (sparse_mask_tc.cu); fast_attention takes it when the rows keep
+// a sizeable share of their causal range.
+bool sparse_mask_preferred(const Shape& s);
+size_t sparse_mask_ws_bytes(const Shape& s);
+bool sparse_mask_supported(const Shape& s, const void* q, const void* k, const void* v);
+cudaError_t sparse_mask_attention(const Shape& s, const void* q, const void* k, const void* v,
+                                  const int32_t* idx, const int32_t* count, void* o, void* ws,
+                                  cudaStream_t st);
+
 // Chunked linear-attention prefill.
 size_t fast_linear_prefill_ws_bytes(const Shape& s);
 bool fast_linear_prefill_supported(const Shape& s, const void* q, const void* k, const void* v);

@@ -1,0 +1,529 @@
+// Sparse softmax attention SA_M over given index rows (lisa_sparse_attn) for
+// many query rows, on the tcgen05 tensor cores (LISA, arXiv 2607.19358v1,
+// Sec. 3.2 Eq. 1: each query head attends over the positions its token's
+// indexer selected; GQA: head h reads KV head h / group).
+//
+// When the rows of a call select a sizeable share of their causal range (a
+// prefill: row t keeps min(M, t+1) of its t+1 positions), gathering every
+// selected row for every query moves the same K/V rows through the SMs over
+// and over.  Here the selections become a bit mask instead, and the attention
+// runs as a flash-attention loop over 128-query x 64-key tiles in which the
+// scores of unselected keys are dropped before the softmax:
+//
+//  k_sel_mask:       one CTA per query row writes the row's selection as bits
+//                    (position s -> bit s) and marks, per 128-row query tile,
+//                    the 64-key tiles that any of its rows selects from.
+//  k_sparse_mask_tc: one CTA per (query tile, query head).  Warp 0 brings Q
+//                    (once) and the K and V tiles of the marked key tiles by
+//                    TMA (128-byte swizzle, 4-stage rings); warp 1 owns TMEM
+//                    and issues S = Q K^T (M = 128 queries, N = 64 keys,
+//                    K = 128 dims) into one of two TMEM score buffers and
+//                    O += P V (M = 128, N = 128 dims, K = 64 keys, V read
+//                    MN-major straight from its TMA tile) into the TMEM
+//                    output; warps 2-5 (one query row per thread, the row's
+//                    TMEM lane) read S, keep only the selected keys, update
+//                    the row's running max and sum (the output is rescaled in
+//                    TMEM only when the max grows by more than 2^8, which
+//                    leaves the result exact), write P as bf16 into shared
+//                    memory in the MMA's swizzled layout, and at the end
+//                    normalise O and store it.
+//
+// Every wait is bounded; one that gives up records LISA_ERR_TIMEOUT, and the
+// kernel waits (bounded) for its own copies and MMAs in flight, releases its
+// TMEM and returns.  Positions outside [0, p] are skipped by k_sel_mask and
+// reported as LISA_ERR_DEVICE_BOUNDS.
+#include <cuda.h>
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "lisa_fast.cuh"
+#include "lisa_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "tma_host.cuh"
+
+namespace lisa {
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kQT = 128;          // query rows per tile (MMA M)
+constexpr int kKT = 64;           // keys per tile
+constexpr int kD = 128;           // head dimension of this path
+constexpr int kStages = 4;        // K (and V) tiles in flight
+constexpr int kThreads = 192;     // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kMaxTiles = 2048;   // key tiles one query tile may visit (keys <= 131072)
+constexpr uint32_t kTries = 1u << 22;
+constexpr float kLazy = 8.0f;     // rescale the output when the max grows by more (log2)
+constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128
+
+struct MaskParams {
+    int T, n_past, M, Lw, nqt, nkw;
+    const int32_t* idx;
+    const int32_t* count;
+    uint32_t* mask;  // [B*T][Lw]: bit s of row (b, t) = position s selected
+    uint32_t* occ;   // [B*nqt][nkw]: bit k = some row of the query tile selects in key tile k
+    unsigned* status;
+};
+
+__global__ void __launch_bounds__(256) k_sel_mask(const MaskParams P) {
+    extern __shared__ uint32_t wbits[];  // the row's Lw words
+    const int row = blockIdx.x, tid = threadIdx.x;
+    const int b = row / P.T, t = row % P.T, p = P.n_past + t;
+    for (int i = tid; i < P.Lw; i += 256) wbits[i] = 0u;
+    __syncthreads();
+    const int cnt = max(0, min(P.count[row], P.M));
+    const int32_t* ix = P.idx + (int64_t)row * P.M;
+    bool bad = false;
+    for (int i = tid; i < cnt; i += 256) {
+        const int pos = ix[i];
+        if (pos < 0 || pos > p) {
+            bad = true;
+            continue;
+        }
+        atomicOr(wbits + (pos >> 5), 1u << (pos & 31));
+    }
+    if (bad) record_error(P.status, kDevBounds);
+    __syncthreads();
+    // the row out, two words (one 64-key tile) per thread and step; the
+    // tiles that hold a selection are OR-ed into the query tile's marks
+    const int ntile = P.Lw / 2;
+    uint2* dst = reinterpret_cast<uint2*>(P.mask + (int64_t)row * P.Lw);
+    const uint2* src = reinterpret_cast<const uint2*>(wbits);
+    uint32_t* occ = P.occ + ((int64_t)b * P.nqt + t / kQT) * P.nkw;
+    for (int i0 = 0; i0 < ntile; i0 += 256) {
+        const int i = i0 + tid;
+        bool any = false;
+        if (i < ntile) {
+            const uint2 v = src[i];
+            dst[i] = v;
+            any = (v.x | v.y) != 0u;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, any);
+        if ((tid & 31) == 0 && bal) atomicOr(occ + (i0 + (tid & ~31)) / 32, bal);
+    }
+}
+
+struct AttnParams {
+    int B, T, H_q, group, nqt, Lw, nkw;
+    float scale_log2;
+    const uint32_t* mask;
+    const uint32_t* occ;
+    bf16* o;
+    unsigned* status;
+};
+
+struct Smem {
+    static constexpr int q = 0;                                  // 2 boxes of 64 dims x 128 rows
+    static constexpr int k = q + 2 * 16384;                      // kStages x (2 x 64 dims x 64 keys)
+    static constexpr int v = k + kStages * 16384;                // the same for V
+    static constexpr int p = v + kStages * 16384;                // 128 rows x 64 keys bf16
+    static constexpr int list = p + 16384;                       // int[kMaxTiles]
+    static constexpr int bars = list + kMaxTiles * 4;            // mbarriers
+    static constexpr int misc = bars + 32 * 8;                   // tmem base, tile count, fail
+    static constexpr int total = misc + 64 + 1024;               // + base alignment slack
+};
+static_assert(Smem::total <= 227 * 1024, "shared memory per CTA");
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+    return ptx::mbar_wait_bounded(bar, parity, kTries);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_sparse_mask_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, const AttnParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* qs = base + Smem::q;
+    uint8_t* ks = base + Smem::k;
+    uint8_t* vs = base + Smem::v;
+    uint8_t* ps = base + Smem::p;
+    int* list = reinterpret_cast<int*>(base + Smem::list);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + Smem::bars);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* k_empty = k_full + kStages;
+    uint64_t* v_full = k_empty + kStages;
+    uint64_t* v_empty = v_full + kStages;
+    uint64_t* s_full = v_empty + kStages;   // [2]
+    uint64_t* s_empty = s_full + 2;         // [2]
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* pv_done = p_full + 1;
+    uint64_t* mma_all = pv_done + 1;        // every MMA this CTA issued has completed
+    uint32_t* misc = reinterpret_cast<uint32_t*>(base + Smem::misc);  // [0] tmem, [1] tiles, [2] fail
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // longest query tiles first; the heads of one query tile run side by side
+    // (they read the same K/V tiles)
+    const int per_qt = P.B * P.H_q;
+    const int qt = P.nqt - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = blockIdx.x % per_qt;
+    const int b = rem / P.H_q, h = rem % P.H_q, g = h / P.group;
+    const int q0 = qt * kQT;
+
+    if (tid == 0) {
+        ptx::mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&k_full[s], 1);
+            ptx::mbar_init(&k_empty[s], 1);
+            ptx::mbar_init(&v_full[s], 1);
+            ptx::mbar_init(&v_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&s_full[s], 1);
+            ptx::mbar_init(&s_empty[s], 4);
+        }
+        ptx::mbar_init(p_full, 4);
+        ptx::mbar_init(pv_done, 1);
+        ptx::mbar_init(mma_all, 1);
+        ptx::fence_mbar_init();
+        misc[2] = 0u;
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(misc, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0) {
+        // the marked key tiles of this query tile, in ascending order
+        const uint32_t* oc = P.occ + ((int64_t)b * P.nqt + qt) * P.nkw;
+        int done = 0;
+        for (int w0 = 0; w0 < P.nkw; w0 += 32) {
+            const uint32_t word = (w0 + lane < P.nkw) ? __ldg(oc + w0 + lane) : 0u;
+            const int c = __popc(word);
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int at = done + incl - c;
+            uint32_t wv = word;
+            while (wv) {
+                const int bit = __ffs(wv) - 1;
+                wv &= wv - 1;
+                if (at < kMaxTiles) list[at] = (w0 + lane) * 32 + bit;
+                ++at;
+            }
+            done += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) misc[1] = (uint32_t)min(done, kMaxTiles);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const int n = (int)misc[1];
+    const uint32_t t_o = tmem + 128;  // output columns
+
+    if (warp == 0) {
+        if (lane == 0 && n > 0) {
+            // ---- producer
+            bool ok = true;
+            ptx::mbar_arrive_expect_tx(q_full, 2 * 16384);
+            ptx::tma_load_3d(qs, &tmap_q, h * kD, q0, b, q_full);
+            ptx::tma_load_3d(qs + 16384, &tmap_q, h * kD + 64, q0, b, q_full);
+            int issued = 0;
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i % kStages, use = i / kStages;
+                const int key0 = list[i] * kKT;
+                if (use > 0) ok = wait_bar(&k_empty[s], (use - 1) & 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(&k_full[s], 16384);
+                ptx::tma_load_3d(ks + s * 16384, &tmap_k, g * kD, key0, b, &k_full[s]);
+                ptx::tma_load_3d(ks + s * 16384 + 8192, &tmap_k, g * kD + 64, key0, b, &k_full[s]);
+                if (use > 0) ok = wait_bar(&v_empty[s], (use - 1) & 1);
+                if (!ok) {
+                    // the K copies just issued land before the CTA may leave
+                    wait_bar(&k_full[s], use & 1);
+                    break;
+                }
+                ptx::mbar_arrive_expect_tx(&v_full[s], 16384);
+                ptx::tma_load_3d(vs + s * 16384, &tmap_v, g * kD, key0, b, &v_full[s]);
+                ptx::tma_load_3d(vs + s * 16384 + 8192, &tmap_v, g * kD + 64, key0, b, &v_full[s]);
+                issued = i + 1;
+            }
+            if (!ok) {
+                misc[2] = 1u;
+                record_error(P.status, kDevTimeout);
+                // copies still in flight land before the shared memory is released
+                for (int i = max(0, issued - kStages); i < issued; ++i) {
+                    ptx::mbar_wait_bounded(&k_full[i % kStages], (i / kStages) & 1, 1u << 16);
+                    ptx::mbar_wait_bounded(&v_full[i % kStages], (i / kStages) & 1, 1u << 16);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && n > 0) {
+            // ---- MMA issuer
+            const uint32_t idesc_s = ptx::idesc_bf16_f32(kQT, kKT);
+            const uint32_t idesc_pv = ptx::idesc_bf16_f32_bmn(kQT, kD);
+            const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs), qd1 = ptx::sdesc_kmajor_sw128(qs + 16384);
+            const uint64_t pd = ptx::sdesc_kmajor_sw128(ps);
+            bool ok = wait_bar(q_full, 0);
+            auto issue_s = [&](int i) {
+                const int s = i % kStages, sb = i & 1;
+                ok = ok && wait_bar(&k_full[s], (i / kStages) & 1);
+                if (ok && i >= 2) ok = wait_bar(&s_empty[sb], ((i >> 1) - 1) & 1);
+                if (!ok) return;
+                ptx::tc_fence_after();
+                const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
+                const uint64_t kd1 = ptx::sdesc_kmajor_sw128(ks + s * 16384 + 8192);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                    const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
+                    ptx::umma_f16(tmem + (uint32_t)(sb * kKT), a, bd, idesc_s, kk > 0);
+                }
+                ptx::umma_commit(&k_empty[s]);
+                ptx::umma_commit(&s_full[sb]);
+            };
+            issue_s(0);
+            for (int i = 0; i < n && ok; ++i) {
+                if (i + 1 < n) issue_s(i + 1);
+                const int s = i % kStages;
+                ok = ok && wait_bar(p_full, i & 1);
+                ok = ok && wait_bar(&v_full[s], (i / kStages) & 1);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    ptx::umma_f16(t_o, pd + 2 * kk, vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
+                                  (i > 0 || kk > 0) ? 1u : 0u);
+                ptx::umma_commit(&v_empty[s]);
+                ptx::umma_commit(pv_done);
+            }
+            if (!ok) {
+                misc[2] = 1u;
+                record_error(P.status, kDevTimeout);
+            }
+            // every MMA issued has completed before TMEM is released
+            ptx::umma_commit(mma_all);
+            ptx::mbar_wait_bounded(mma_all, 0, kTries);
+        }
+    } else {
+        // ---- softmax: thread = query row (its TMEM lane)
+        const int lb = (warp & 3) * 32;
+        const int r = lb + lane;
+        const int t = q0 + r;
+        const bool valid = t < P.T;
+        const uint32_t* mrow = P.mask + ((int64_t)b * P.T + (valid ? t : 0)) * P.Lw;
+        const uint32_t t_row = tmem + ((uint32_t)lb << 16);
+        float m_used = -INFINITY, l = 0.0f;
+        uint2 mk_next = make_uint2(0u, 0u);
+        if (valid && n > 0) mk_next = __ldg(reinterpret_cast<const uint2*>(mrow) + list[0]);
+        int pv_waited = 0;  // PV products known complete
+        bool ok = true;
+        for (int i = 0; i < n; ++i) {
+            const int sb = i & 1;
+            const uint2 mk = mk_next;
+            if (valid && i + 1 < n) mk_next = __ldg(reinterpret_cast<const uint2*>(mrow) + list[i + 1]);
+            // (waits agree across the warp: the TMEM accesses that follow are collective)
+            if (!__all_sync(0xffffffffu, wait_bar(&s_full[sb], (i >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            uint32_t sr[64];
+            ptx::tmem_ld32(t_row + (uint32_t)(sb * kKT), *reinterpret_cast<uint32_t(*)[32]>(sr));
+            ptx::tmem_ld32(t_row + (uint32_t)(sb * kKT + 32), *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+            ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
+            // the tile's largest selected score (the scale is positive)
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+                const uint32_t w = k < 32 ? mk.x : mk.y;
+                if ((w >> (k & 31)) & 1u) mx = fmaxf(mx, __uint_as_float(sr[k]));
+            }
+            mx = mx == -INFINITY ? -INFINITY : mx * P.scale_log2;
+            // the running max moves when a selected score exceeds it by more
+            // than 2^kLazy (the output and sum are rescaled then), or when the
+            // row meets its first selected key (the output is still zero)
+            const bool first = m_used == -INFINITY && mx != -INFINITY;
+            const bool grow = m_used != -INFINITY && mx > m_used + kLazy;
+            if (__any_sync(0xffffffffu, grow)) {
+                // the output must hold every product so far before it is rescaled
+                if (i > 0 && pv_waited < i) {
+                    if (!__all_sync(0xffffffffu, wait_bar(pv_done, (i - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    pv_waited = i;
+                }
+                ptx::tc_fence_after();
+                const float alpha = grow ? exp2f(m_used - mx) : 1.0f;
+#pragma unroll 1
+                for (int c = 0; c < kD; c += 32) {
+                    uint32_t ov[32];
+                    ptx::tmem_ld32(t_row + 128 + (uint32_t)c, ov);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    ptx::tmem_st32(t_row + 128 + (uint32_t)c, ov);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                l *= alpha;
+            }
+            if (first || grow) m_used = mx;
+            // probabilities of the selected keys (bf16 pairs), zero elsewhere
+            uint32_t pk[32];
+            float lsum = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 64; k += 2) {
+                const uint32_t w = k < 32 ? mk.x : mk.y;
+                const bool s0 = (w >> (k & 31)) & 1u, s1 = (w >> ((k + 1) & 31)) & 1u;
+                const float p0 = s0 ? exp2f(fmaf(__uint_as_float(sr[k]), P.scale_log2, -m_used)) : 0.0f;
+                const float p1 = s1 ? exp2f(fmaf(__uint_as_float(sr[k + 1]), P.scale_log2, -m_used)) : 0.0f;
+                lsum += p0 + p1;
+                pk[k >> 1] = ptx::pack_bf16(p0, p1);
+            }
+            l += lsum;
+            // the P tile is free once the previous product has read it
+            if (i > 0 && pv_waited < i) {
+                if (!__all_sync(0xffffffffu, wait_bar(pv_done, (i - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                pv_waited = i;
+            }
+            // row r of P: 128 bytes, 16-byte chunk c at chunk c ^ (r % 8)
+            uint8_t* prow = ps + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            ptx::fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(p_full);
+        }
+        if (!ok) {
+            misc[2] = 1u;
+            if (lane == 0) record_error(P.status, kDevTimeout);
+        }
+        // ---- epilogue: O / l, bf16, to global memory
+        bf16* orow = P.o + (((int64_t)b * P.T + (valid ? t : 0)) * P.H_q + h) * kD;
+        const bool have = __all_sync(0xffffffffu, ok && n > 0 && wait_bar(pv_done, (n - 1) & 1));
+        if (have) ptx::tc_fence_after();
+        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < kD; c += 32) {
+            uint32_t ov[32];
+            if (have) {
+                ptx::tmem_ld32(t_row + 128 + (uint32_t)c, ov);
+                ptx::tmem_ld_wait();
+            }
+            uint32_t pkd[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                pkd[e] = have ? ptx::pack_bf16(__uint_as_float(ov[2 * e]) * inv,
+                                               __uint_as_float(ov[2 * e + 1]) * inv)
+                              : 0u;
+            if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+struct MaskLayout {
+    int Lw, nqt, nkw;
+    size_t mask, occ, end;
+};
+
+MaskLayout mask_layout(const Shape& s) {
+    MaskLayout m;
+    m.Lw = (s.L + kKT - 1) / kKT * 2;           // 2 words per 64-key tile
+    m.nqt = (s.T + kQT - 1) / kQT;
+    m.nkw = (m.Lw / 2 + 31) / 32;
+    m.mask = kStatusBytes;
+    m.occ = m.mask + (((size_t)s.B * s.T * m.Lw * 4 + 255) & ~(size_t)255);
+    m.end = m.occ + (((size_t)s.B * m.nqt * m.nkw * 4 + 255) & ~(size_t)255);
+    return m;
+}
+
+}  // namespace
+
+// The masked tensor-core form pays for every key of a visited 64-key tile,
+// the gather form for every selected key of every row: prefer the first when
+// the rows keep a sizeable share of their causal range.  The estimate assumes
+// min(M, p + 1) selected positions per row (what lisa_topm writes).
+bool sparse_mask_preferred(const Shape& s) {
+    if (s.dtype != LISA_BF16 || s.d != kD || s.T < kQT) return false;
+    if (s.L > kMaxTiles * kKT) return false;
+    double sel = 0.0, causal = 0.0;
+    for (int t = 0; t < s.T; t += 16) {  // every 16th row is plenty for the ratio
+        const double p1 = (double)s.n_past + t + 1;
+        sel += std::min((double)s.M, p1);
+        causal += p1;
+    }
+    return sel >= causal / 16.0;
+}
+
+size_t sparse_mask_ws_bytes(const Shape& s) { return mask_layout(s).end; }
+
+bool sparse_mask_supported(const Shape& s, const void* q, const void* k, const void* v) {
+    if (!sparse_mask_preferred(s)) return false;
+    if (!(aligned16(q) && aligned16(k) && aligned16(v))) return false;
+    return tma_encode_fn() != nullptr;
+}
+
+cudaError_t sparse_mask_attention(const Shape& s, const void* q, const void* k, const void* v,
+                                  const int32_t* idx, const int32_t* count, void* o, void* ws,
+                                  cudaStream_t st) {
+    const MaskLayout lay = mask_layout(s);
+    char* w8 = static_cast<char*>(ws);
+    uint32_t* mask = reinterpret_cast<uint32_t*>(w8 + lay.mask);
+    uint32_t* occ = reinterpret_cast<uint32_t*>(w8 + lay.occ);
+    cudaError_t e = cudaMemsetAsync(occ, 0, (size_t)s.B * lay.nqt * lay.nkw * 4, st);
+    if (e != cudaSuccess) return e;
+
+    MaskParams mp;
+    mp.T = s.T; mp.n_past = s.n_past; mp.M = s.M; mp.Lw = lay.Lw; mp.nqt = lay.nqt; mp.nkw = lay.nkw;
+    mp.idx = idx; mp.count = count; mp.mask = mask; mp.occ = occ; mp.status = static_cast<unsigned*>(ws);
+    k_sel_mask<<<s.B * s.T, 256, (size_t)lay.Lw * 4, st>>>(mp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    CUtensorMap tq, tk, tv;
+    memset(&tq, 0, sizeof(tq));
+    memset(&tk, 0, sizeof(tk));
+    memset(&tv, 0, sizeof(tv));
+    const uint64_t qrow = (uint64_t)s.H_q * kD, kvrow = (uint64_t)s.H_kv * kD;
+    if (!make_tmap_bf16_3d(&tq, q, qrow, s.T, s.B, qrow, (uint64_t)s.T * qrow, 64, kQT) ||
+        !make_tmap_bf16_3d(&tk, k, kvrow, s.L, s.B, kvrow, (uint64_t)s.N_max * kvrow, 64, kKT) ||
+        !make_tmap_bf16_3d(&tv, v, kvrow, s.L, s.B, kvrow, (uint64_t)s.N_max * kvrow, 64, kKT))
+        return cudaErrorInvalidValue;
+
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+        e = cudaFuncSetAttribute(k_sparse_mask_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Smem::total);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    AttnParams ap;
+    ap.B = s.B; ap.T = s.T; ap.H_q = s.H_q; ap.group = s.group; ap.nqt = lay.nqt; ap.Lw = lay.Lw;
+    ap.nkw = lay.nkw; ap.scale_log2 = s.sm_scale * 1.4426950408889634f;
+    ap.mask = mask; ap.occ = occ; ap.o = static_cast<bf16*>(o); ap.status = static_cast<unsigned*>(ws);
+    k_sparse_mask_tc<<<s.B * lay.nqt * s.H_q, kThreads, Smem::total, st>>>(tq, tk, tv, ap);
+    return cudaGetLastError();
+}
+
+}  // namespace lisa

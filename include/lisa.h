@@ -144,8 +144,15 @@ LISA_API lisa_status lisa_topm(const lisa_dims* dims, const void* q_I, const voi
 /* Sparse softmax attention SA_M (Sec. 3.2, Eq. 1) of each query head over the
  * count[b,t] positions in idx[b,t,:] (any order; entries past count ignored):
  *   o_sparse[h] = softmax_s(sm_scale * <q[h], K[s,g]>) . V[s,g],  g = h / (H_q/H_kv)
- * Positions outside [0, p] are skipped and reported as LISA_ERR_DEVICE_BOUNDS
- * through the status word.  count == 0 gives a zero output. */
+ * The positions of a row are a set: they must be distinct (lisa_topm and
+ * lisa_window_indices write distinct positions); a repeated position may
+ * count once or twice.  Positions outside [0, p] are skipped and reported as
+ * LISA_ERR_DEVICE_BOUNDS through the status word.  count == 0 gives a zero
+ * output.  Calls whose rows keep a sizeable share of their causal range (a
+ * prefill) run as masked tensor-core tiles over the key tiles the rows select
+ * from; others gather each selected row.  Workspace:
+ * lisa_workspace_size(.., LISA_OP_SPARSE_ATTN) (the selection mask, about
+ * B*T*(n_past+T)/8 bytes, for the first form). */
 LISA_API lisa_status lisa_sparse_attn(const lisa_dims* dims, const void* q, const void* k_cache,
                              const void* v_cache, const int32_t* idx, const int32_t* count,
                              void* o_sparse, void* ws, size_t ws_bytes, void* stream);
