@@ -7,19 +7,22 @@
 // (elu+1 mode: the same for the normaliser, z_c = z_{c-1} + sum phi(K_c), and
 // O_c is divided row-wise by phi(Q_c) z_{c-1} + rowsum(tril(phi(Q_c) phi(K_c)^T)).)
 //
-// k_la_chunk_sums  (B x H_kv x chunks CTAs): U_c = phi(K_c)^T V_c in fp32
-//                   (mma m16n8k16, bf16 operands), and sum_t phi(K_c) for z.
-// k_la_prefix      (one thread per state element): U_c <- S_0 + sum_{c'<c} U_c'
-//                   in place; the final state goes to S (and z).
-// k_la_chunk_out   (B x H_kv x chunks CTAs, two query heads at a time): the
-//                   inter-chunk term uses the fp32 prefix state split into two
-//                   bf16 halves (hi + lo), so it keeps ~16 bits of mantissa;
-//                   the intra-chunk term applies the inclusive causal mask.
+// k_la_sums_tc  (B x H_kv x chunks CTAs): U_c = phi(K_c)^T V_c on tcgen05,
+//               operands by TMA, accumulator in TMEM; sum_t phi(K_c) for z.
+// k_la_prefix   (one thread per state element): U_c <- S_0 + sum_{c'<c} U_c'
+//               in place; the final state goes to S (and z).
+// k_la_out_tc   (B x H_kv x chunks CTAs): every product of the chunk's query
+//               heads on tcgen05, the inter-chunk term through the fp32 prefix
+//               state split into two bf16 halves (hi + lo, ~16 bits kept).
+// Every wait is bounded; one that gives up records LISA_ERR_TIMEOUT.
+#include <cuda.h>
 #include <math.h>
+#include <string.h>
 
 #include "lisa_fast.cuh"
 #include "lisa_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "tma_host.cuh"
 
 namespace lisa {
 namespace {
@@ -28,7 +31,7 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kD = 128;
 constexpr int kC = 64;                 // chunk length of this path
-constexpr int kRow = kD * 2 + 16;      // padded shared-memory row (bytes) of 128 bf16
+constexpr uint32_t kTries = 1u << 22;  // polls of a bounded wait
 
 struct LaParams {
     int B, T, H_q, H_kv, group, phi, nch;
@@ -40,103 +43,125 @@ struct LaParams {
     bf16* o;
     float* U;      // workspace [B][H_kv][nch][128][128]
     float* Z;      // workspace [B][H_kv][nch][128]
+    unsigned* status;
 };
 
-__device__ __forceinline__ float feat(int phi, float x) {
-    if (phi == LISA_PHI_IDENTITY) return x;
-    return x > 0.0f ? x + 1.0f : __expf(x);
-}
-
-// Loads rows [t0, t0 + 64) of one head (row stride `stride` elements) into
-// padded shared memory as bf16 (rows past T are zero).  mode 0: values as
-// given; 1: phi(x); 2: phi(x) - 1, which bf16 holds far more accurately than
-// phi(x) itself in the elu+1 map (phi(x) is close to 1 for small x).
-__device__ __forceinline__ void load_rows(uint8_t* dst, const bf16* src, int64_t stride, int t0,
-                                          int T, int phi, int mode, int nthreads) {
-    for (int e = threadIdx.x; e < kC * (kD / 8); e += nthreads) {
-        const int r = e / (kD / 8), c8 = e % (kD / 8);
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        const bool valid = t0 + r < T;
-        if (valid) u = *reinterpret_cast<const uint4*>(src + (int64_t)(t0 + r) * stride + c8 * 8);
-        if (mode != 0 && phi != LISA_PHI_IDENTITY && valid) {
-            const float sub = mode == 2 ? 1.0f : 0.0f;
-            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float2 f = __bfloat1622float2(h2[x]);
-                const float a = f.x > 0.0f ? f.x + (1.0f - sub) : (mode == 2 ? expm1f(f.x) : __expf(f.x));
-                const float c = f.y > 0.0f ? f.y + (1.0f - sub) : (mode == 2 ? expm1f(f.y) : __expf(f.y));
-                h2[x] = __floats2bfloat162_rn(a, c);
-            }
-        }
-        *reinterpret_cast<uint4*>(dst + r * kRow + c8 * 16) = u;
-    }
-}
-
 // ---------------------------------------------------------------- chunk sums
-__global__ void __launch_bounds__(256) k_la_chunk_sums(const LaParams P) {
-    __shared__ __align__(128) uint8_t ks[kC * kRow];
-    __shared__ __align__(128) uint8_t vs[kC * kRow];
+// One CTA per (sequence, KV head, chunk): U_c = phi(K_c)^T V_c on the tensor
+// cores, M = 128 key features x N = 128 value dims x K = 64 tokens, both
+// operands MN-major straight from their TMA tiles (128-byte swizzle).  In the
+// elu+1 mode the tile holds phi(K) - 1 (bf16 keeps it far more accurately
+// than phi(K), which is near 1 for small keys) and the rank-one rest,
+// 1 (x) sum_t V[t], is added in the epilogue; the chunk's sum of phi(k) goes
+// to Z.  Thread i reads TMEM lane i (key feature i) and writes row i of U_c.
+constexpr int kSumThreads = 128;
+
+__device__ __forceinline__ float elu1_minus1(float x) { return x > 0.0f ? x : expm1f(x); }
+
+// Element (t, c) of a [64 rows][128 cols] bf16 tile held as two TMA boxes of
+// 64 columns (128-byte rows, 128-byte swizzle), box b at byte b * 8192.
+__device__ __forceinline__ int sw_off64(int t, int c) {
+    const int box = c >> 6, cc = c & 63;
+    return box * 8192 + t * 128 + ((((cc >> 3) ^ (t & 7)) << 4) | ((cc & 7) << 1));
+}
+
+__global__ void __launch_bounds__(kSumThreads, 1)
+    k_la_sums_tc(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                 const LaParams P) {
+    __shared__ __align__(1024) uint8_t ks[16384];
+    __shared__ __align__(1024) uint8_t vs[16384];
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ uint32_t tmem_slot;
+    __shared__ float vsum[kD];
     const int c = blockIdx.x % P.nch, g = (blockIdx.x / P.nch) % P.H_kv, b = blockIdx.x / (P.nch * P.H_kv);
     const int t0 = c * kC;
-    const int64_t rs = (int64_t)P.H_kv * kD;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const bool norm = P.phi == LISA_PHI_ELU1_NORM;
-    // elu+1: the tensor cores see phi(K) - 1; U = (phi(K) - 1)^T V + 1 (x) sum_t V[t]
-    load_rows(ks, P.k + ((int64_t)b * P.T * P.H_kv + g) * kD, rs, t0, P.T, P.phi, 2, 256);
-    load_rows(vs, P.v + ((int64_t)b * P.T * P.H_kv + g) * kD, rs, t0, P.T, P.phi, 0, 256);
-    __shared__ float vsum[kD];
+    if (tid == 0) {
+        ptx::mbar_init(&bars[0], 1);
+        ptx::mbar_init(&bars[1], 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&tmem_slot, 128);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
     __syncthreads();
-    if (norm && threadIdx.x < kD) {
-        float a = 0.0f;
-        for (int t = 0; t < kC; ++t)
-            a += __bfloat162float(*reinterpret_cast<const bf16*>(vs + t * kRow + threadIdx.x * 2));
-        vsum[threadIdx.x] = a;
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(&bars[0], 32768);
+        ptx::tma_load_3d(ks, &tmap_k, g * kD, t0, b, &bars[0]);
+        ptx::tma_load_3d(ks + 8192, &tmap_k, g * kD + 64, t0, b, &bars[0]);
+        ptx::tma_load_3d(vs, &tmap_v, g * kD, t0, b, &bars[0]);
+        ptx::tma_load_3d(vs + 8192, &tmap_v, g * kD + 64, t0, b, &bars[0]);
+    }
+    bool ok = __syncthreads_and(ptx::mbar_wait_bounded(&bars[0], 0, kTries));
+    const int nvalid = min(kC, P.T - t0);
+    float zsum = 0.0f;
+    if (ok && norm) {
+        // phi(K) - 1 in place (rows past T stay zero), the sum of V per value
+        // dim and of phi(k) per key feature (thread = column)
+        __nv_bfloat162* kw = reinterpret_cast<__nv_bfloat162*>(ks);
+        for (int e = tid; e < 16384 / 4; e += kSumThreads) {
+            const int t = ((e * 4) & 8191) >> 7;  // the token row of this word
+            if (t < nvalid) {
+                const float2 f = __bfloat1622float2(kw[e]);
+                kw[e] = __floats2bfloat162_rn(elu1_minus1(f.x), elu1_minus1(f.y));
+            }
+        }
+        float vs_acc = 0.0f;
+        for (int t = 0; t < nvalid; ++t)
+            vs_acc += __bfloat162float(*reinterpret_cast<const bf16*>(vs + sw_off64(t, tid)));
+        vsum[tid] = vs_acc;
+        __syncthreads();
+        for (int t = 0; t < nvalid; ++t)
+            zsum += __bfloat162float(*reinterpret_cast<const bf16*>(ks + sw_off64(t, tid)));
+        zsum += (float)nvalid;
+        ptx::fence_proxy_async_shared();
     }
     __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gid = lane >> 2, tq = lane & 3;
-    const int m0 = warp * 16;  // key-feature rows of this warp
-    float acc[16][4];
+    if (tid == 0 && ok) {
+        ptx::tc_fence_after();
+        // A = phi(K)^T: M = features (contiguous within a box), K = tokens;
+        // B = V: N = value dims (contiguous), K = tokens
+        const uint32_t idesc = ptx::idesc_bf16_f32_bmn(kD, kD) | (1u << 15);
+        const uint64_t ad = ptx::sdesc_mnmajor_sw128(ks, 8192, 1024);
+        const uint64_t bd = ptx::sdesc_mnmajor_sw128(vs, 8192, 1024);
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
+        for (int kk = 0; kk < kC / 16; ++kk)
+            ptx::umma_f16(tmem, ad + (uint64_t)(128 * kk), bd + (uint64_t)(128 * kk), idesc, kk > 0);
+        ptx::umma_commit(&bars[1]);
+    }
+    ok = ok && __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&bars[1], 0, kTries));
+    if (!ok) {
+        if ((tid & 31) == 0) record_error(P.status, kDevTimeout);
+    } else {
+        ptx::tc_fence_after();
+        const int lb = warp * 32, i = lb + (tid & 31);
+        float* U = P.U + (((int64_t)b * P.H_kv + g) * P.nch + c) * kD * kD + (int64_t)i * kD;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tmem + ((uint32_t)lb << 16) + (uint32_t)c0, r);
+            ptx::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[n][e] = 0.0f;
-    const uint32_t kb = ptx::smem_u32(ks), vb = ptx::smem_u32(vs);
-#pragma unroll
-    for (int kt = 0; kt < kC / 16; ++kt) {
-        // A = phi(K)^T (rows = features, cols = tokens) from K rows via transposed ldmatrix
-        uint32_t a[4];
-        {
-            const int j = lane >> 3;
-            const int t = kt * 16 + (j >> 1) * 8 + (lane & 7);
-            const int f = m0 + (j & 1) * 8;
-            ptx::ldmatrix_x4_trans(a, kb + t * kRow + f * 2);
+            for (int e = 0; e < 32; e += 4) {
+                float4 u;
+                u.x = __uint_as_float(r[e]) + (norm ? vsum[c0 + e] : 0.0f);
+                u.y = __uint_as_float(r[e + 1]) + (norm ? vsum[c0 + e + 1] : 0.0f);
+                u.z = __uint_as_float(r[e + 2]) + (norm ? vsum[c0 + e + 2] : 0.0f);
+                u.w = __uint_as_float(r[e + 3]) + (norm ? vsum[c0 + e + 3] : 0.0f);
+                *reinterpret_cast<float4*>(U + c0 + e) = u;
+            }
         }
-#pragma unroll
-        for (int n = 0; n < 16; n += 2) {
-            uint32_t vr[4];
-            const int t = kt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-            const int f = (n + (lane >> 4)) * 8;
-            ptx::ldmatrix_x4_trans(vr, vb + t * kRow + f * 2);
-            ptx::mma_bf16(acc[n], a, vr[0], vr[1]);
-            ptx::mma_bf16(acc[n + 1], a, vr[2], vr[3]);
-        }
+        if (norm) P.Z[(((int64_t)b * P.H_kv + g) * P.nch + c) * kD + tid] = zsum;
     }
-    float* U = P.U + (((int64_t)b * P.H_kv + g) * P.nch + c) * kD * kD;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int col = n * 8 + 2 * tq;
-        const float r0 = norm ? vsum[col] : 0.0f, r1 = norm ? vsum[col + 1] : 0.0f;
-        *reinterpret_cast<float2*>(U + (m0 + gid) * kD + col) = make_float2(acc[n][0] + r0, acc[n][1] + r1);
-        *reinterpret_cast<float2*>(U + (m0 + gid + 8) * kD + col) = make_float2(acc[n][2] + r0, acc[n][3] + r1);
-    }
-    if (norm && threadIdx.x < kD) {
-        // sum_t phi(k_t) = sum_t (phi(k_t) - 1) + (valid tokens of the chunk)
-        float zs = (float)min(kC, P.T - t0);
-        for (int t = 0; t < kC; ++t)
-            zs += __bfloat162float(*reinterpret_cast<const bf16*>(ks + t * kRow + threadIdx.x * 2));
-        P.Z[(((int64_t)b * P.H_kv + g) * P.nch + c) * kD + threadIdx.x] = zs;
-    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 0) ptx::tmem_dealloc(tmem, 128);
 }
 
 // ---------------------------------------------------------------- prefix over chunks
@@ -180,165 +205,321 @@ __global__ void __launch_bounds__(256) k_la_prefix(const LaParams P) {
 }
 
 // ---------------------------------------------------------------- chunk outputs
-struct OutSmem {
-    static constexpr int shi = 0;                      // S_{c-1} high half, bf16 [128][128]
-    static constexpr int slo = shi + kD * kRow;        // low half
-    static constexpr int k = slo + kD * kRow;          // phi(K_c) [64][128]
-    static constexpr int v = k + kC * kRow;            // V_c
-    static constexpr int q = v + kC * kRow;            // phi(Q_c) of two heads [2][64][128]
-    static constexpr int zc = q + 2 * kC * kRow;       // z_{c-1} float[128]
-    static constexpr int total = zc + kD * 4;
-};
+// One CTA per (sequence, KV head, chunk).  The group's query heads go two at a
+// time through 128-row tiles (rows 0-63: the chunk's tokens of head 2m, rows
+// 64-127: of head 2m + 1), all products on the tensor cores with the
+// accumulators in TMEM:
+//   O  = phi(Q) S_hi + phi(Q) S_lo       (M = 128, N = 128, K = 128 features;
+//                                          S_{c-1} split into two bf16 halves,
+//                                          MN-major, so ~16 bits are kept)
+//   Si = phi(Q) phi(K_c)^T                (N = 64 tokens)
+//   O += tril(Si) V_c                     (K = 64 tokens, V MN-major from TMA)
+// Warp 0 brings K_c, V_c and the query tiles by TMA (two query buffers);
+// warp 1 owns TMEM (two O and two Si buffers) and issues the MMAs; warps 2-5
+// (thread = tile row = TMEM lane) write the two halves of S_{c-1}, apply phi
+// in the elu+1 mode, mask Si causally into P (bf16, shared memory), and
+// write O (divided by phi(q) . z_{c-1} + the row sum of tril(Si) in the elu+1
+// mode) as bf16.
+constexpr int kOutThreads = 192;
 
-__global__ void __launch_bounds__(256, 1) k_la_chunk_out(const LaParams P) {
-    extern __shared__ __align__(128) uint8_t la_raw[];
+struct OutSmem {
+    static constexpr int shi = 0;                 // 2 blocks of 128 features x 64 dims (MN-major)
+    static constexpr int slo = shi + 32768;
+    static constexpr int k = slo + 32768;         // K_c: 2 boxes of 64 features x 64 tokens
+    static constexpr int v = k + 16384;           // V_c
+    static constexpr int q = v + 16384;           // 2 buffers x 2 feature halves x 2 heads x 64 rows
+    static constexpr int p = q + 2 * 32768;       // tril(Si): 128 rows x 64 tokens bf16
+    static constexpr int zc = p + 16384;          // z_{c-1}: float[128]
+    static constexpr int bars = zc + 512;
+    static constexpr int misc = bars + 24 * 8;
+    static constexpr int total = misc + 16 + 1024;
+};
+static_assert(OutSmem::total <= 227 * 1024, "shared memory per CTA");
+
+__device__ __forceinline__ void phi_inplace(uint8_t* buf, int bytes, int lt, int nt) {
+    __nv_bfloat162* w = reinterpret_cast<__nv_bfloat162*>(buf);
+    for (int e = lt; e < bytes / 4; e += nt) {
+        const float2 f = __bfloat1622float2(w[e]);
+        w[e] = __floats2bfloat162_rn(f.x > 0.0f ? f.x + 1.0f : __expf(f.x),
+                                     f.y > 0.0f ? f.y + 1.0f : __expf(f.y));
+    }
+}
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+    k_la_out_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                const __grid_constant__ CUtensorMap tmap_v, const LaParams P) {
+    extern __shared__ uint8_t la_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(la_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* shi = base + OutSmem::shi;
+    uint8_t* slo = base + OutSmem::slo;
+    uint8_t* kt = base + OutSmem::k;
+    uint8_t* vt = base + OutSmem::v;
+    uint8_t* qb = base + OutSmem::q;
+    uint8_t* pt = base + OutSmem::p;
+    float* zc = reinterpret_cast<float*>(base + OutSmem::zc);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + OutSmem::bars);
+    uint64_t* kv_full = bars;        // K_c and V_c landed
+    uint64_t* q_full = bars + 1;     // [2]
+    uint64_t* q_empty = bars + 3;    // [2]
+    uint64_t* s_ready = bars + 5;    // S halves written, phi applied to K_c (4 warps)
+    uint64_t* q_ready = bars + 6;    // [2] phi applied to the query tile (4 warps)
+    uint64_t* si_full = bars + 8;    // [2]
+    uint64_t* p_full = bars + 10;    // 4 warps
+    uint64_t* o_full = bars + 11;    // [2]
+    uint64_t* o_empty = bars + 13;   // [2] (4 warps)
+    uint64_t* mma_all = bars + 15;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(base + OutSmem::misc);
+
     const int c = blockIdx.x % P.nch, g = (blockIdx.x / P.nch) % P.H_kv, b = blockIdx.x / (P.nch * P.H_kv);
     const int t0 = c * kC;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int gid = lane >> 2, tq = lane & 3;
     const bool norm = P.phi == LISA_PHI_ELU1_NORM;
-    // prefix state of this chunk, split into bf16 hi + lo
-    const float* Sp = P.U + (((int64_t)b * P.H_kv + g) * P.nch + c) * kD * kD;
-    for (int e = tid; e < kD * kD / 2; e += 256) {
-        const int r = e / (kD / 2), c2 = (e % (kD / 2)) * 2;
-        const float2 f = *reinterpret_cast<const float2*>(Sp + r * kD + c2);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(f.x, f.y);
-        const float2 hf = __bfloat1622float2(hi);
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(f.x - hf.x, f.y - hf.y);
-        *reinterpret_cast<__nv_bfloat162*>(la_raw + OutSmem::shi + r * kRow + c2 * 2) = hi;
-        *reinterpret_cast<__nv_bfloat162*>(la_raw + OutSmem::slo + r * kRow + c2 * 2) = lo;
+    const int n_mt = (P.group + 1) / 2;  // 128-row tiles (two heads each)
+
+    if (tid == 0) {
+        ptx::mbar_init(kv_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&q_full[i], 1);
+            ptx::mbar_init(&q_empty[i], 1);
+            ptx::mbar_init(&q_ready[i], 4);
+            ptx::mbar_init(&si_full[i], 1);
+            ptx::mbar_init(&o_full[i], 1);
+            ptx::mbar_init(&o_empty[i], 4);
+        }
+        ptx::mbar_init(s_ready, 4);
+        ptx::mbar_init(p_full, 4);
+        ptx::mbar_init(mma_all, 1);
+        ptx::fence_mbar_init();
     }
-    const int64_t rs_kv = (int64_t)P.H_kv * kD;
-    load_rows(la_raw + OutSmem::k, P.k + ((int64_t)b * P.T * P.H_kv + g) * kD, rs_kv, t0, P.T, P.phi, 1, 256);
-    load_rows(la_raw + OutSmem::v, P.v + ((int64_t)b * P.T * P.H_kv + g) * kD, rs_kv, t0, P.T, P.phi, 0, 256);
-    float* zc = reinterpret_cast<float*>(la_raw + OutSmem::zc);
-    if (norm && tid < kD) zc[tid] = P.Z[(((int64_t)b * P.H_kv + g) * P.nch + c) * kD + tid];
-    const uint32_t shi = ptx::smem_u32(la_raw + OutSmem::shi), slo = ptx::smem_u32(la_raw + OutSmem::slo);
-    const uint32_t kbase = ptx::smem_u32(la_raw + OutSmem::k), vbase = ptx::smem_u32(la_raw + OutSmem::v);
-    const int half = warp >> 2;          // which of the two heads
-    const int r0 = (warp & 3) * 16;      // query rows of this warp within the chunk
-    const int64_t rs_q = (int64_t)P.H_q * kD;
-    for (int hp = 0; hp < P.group; hp += 2) {
-        __syncthreads();  // previous pair finished with the query buffer
-        for (int x = 0; x < 2; ++x)
-            if (hp + x < P.group)
-                load_rows(la_raw + OutSmem::q + x * kC * kRow,
-                          P.q + ((int64_t)b * P.T * P.H_q + g * P.group + hp + x) * kD, rs_q, t0,
-                          P.T, P.phi, 1, 256);
-        __syncthreads();
-        const int h = hp + half;
-        if (h >= P.group) continue;
-        const uint32_t qb = ptx::smem_u32(la_raw + OutSmem::q + half * kC * kRow);
-        float o[16][4];
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[n][e] = 0.0f;
-        float sc[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[n][e] = 0.0f;
-        float qz[2] = {0.0f, 0.0f};  // phi(q) . z_{c-1} of rows gid, gid + 8
-#pragma unroll 2
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            uint32_t a[4];
-            {
-                const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int col = ks * 16 + (lane >> 4) * 8;
-                ptx::ldmatrix_x4(a, qb + row * kRow + col * 2);
-            }
-            // inter-chunk: phi(Q) S_{c-1}, both halves of S
-#pragma unroll
-            for (int n = 0; n < 16; n += 2) {
-                uint32_t br[4];
-                const int kr = ks * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                const int col = (n + (lane >> 4)) * 8;
-                ptx::ldmatrix_x4_trans(br, shi + kr * kRow + col * 2);
-                ptx::mma_bf16(o[n], a, br[0], br[1]);
-                ptx::mma_bf16(o[n + 1], a, br[2], br[3]);
-                ptx::ldmatrix_x4_trans(br, slo + kr * kRow + col * 2);
-                ptx::mma_bf16(o[n], a, br[0], br[1]);
-                ptx::mma_bf16(o[n + 1], a, br[2], br[3]);
-            }
-            // intra-chunk scores: phi(Q) phi(K)^T over the chunk's 64 keys
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                uint32_t kr2[2];
-                {
-                    uint32_t kr4[4];
-                    const int key = n * 8 + (lane & 7);
-                    const int col = ks * 16 + ((lane >> 3) & 1) * 8;
-                    ptx::ldmatrix_x4(kr4, kbase + key * kRow + col * 2);
-                    kr2[0] = kr4[0];
-                    kr2[1] = kr4[1];
+    if (warp == 1) {
+        ptx::tmem_alloc(misc, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    auto heads_of = [&](int m) { return min(2, P.group - 2 * m); };
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- producer
+            ptx::mbar_arrive_expect_tx(kv_full, 32768);
+            ptx::tma_load_3d(kt, &tmap_k, g * kD, t0, b, kv_full);
+            ptx::tma_load_3d(kt + 8192, &tmap_k, g * kD + 64, t0, b, kv_full);
+            ptx::tma_load_3d(vt, &tmap_v, g * kD, t0, b, kv_full);
+            ptx::tma_load_3d(vt + 8192, &tmap_v, g * kD + 64, t0, b, kv_full);
+            bool ok = true;
+            for (int m = 0; m < n_mt && ok; ++m) {
+                const int qi = m & 1;
+                if (m >= 2) ok = ptx::mbar_wait_bounded(&q_empty[qi], ((m >> 1) - 1) & 1, kTries);
+                if (!ok) break;
+                const int nh = heads_of(m);
+                uint8_t* dst = qb + qi * 32768;
+                ptx::mbar_arrive_expect_tx(&q_full[qi], (uint32_t)nh * 16384);
+                for (int hh = 0; hh < nh; ++hh) {
+                    const int x = (g * P.group + 2 * m + hh) * kD;
+                    ptx::tma_load_3d(dst + hh * 8192, &tmap_q, x, t0, b, &q_full[qi]);
+                    ptx::tma_load_3d(dst + 16384 + hh * 8192, &tmap_q, x + 64, t0, b, &q_full[qi]);
                 }
-                ptx::mma_bf16(sc[n], a, kr2[0], kr2[1]);
             }
+            if (!ok) record_error(P.status, kDevTimeout);
         }
-        if (norm) {
-            // phi(q) . z_{c-1} for rows r0 + gid and r0 + gid + 8, from shared memory
-            const uint8_t* qrow0 = la_raw + OutSmem::q + half * kC * kRow + (r0 + gid) * kRow;
-            const uint8_t* qrow1 = qrow0 + 8 * kRow;
-            for (int f = tq; f < kD; f += 4) {
-                qz[0] = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(qrow0 + f * 2)), zc[f], qz[0]);
-                qz[1] = fmaf(__bfloat162float(*reinterpret_cast<const bf16*>(qrow1 + f * 2)), zc[f], qz[1]);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer
+            const uint32_t id_qs = ptx::idesc_bf16_f32_bmn(128, kD);
+            const uint32_t id_qk = ptx::idesc_bf16_f32(128, kC);
+            const uint32_t id_pv = ptx::idesc_bf16_f32_bmn(128, kD);
+            const uint64_t shd = ptx::sdesc_mnmajor_sw128(shi, 16384, 1024);
+            const uint64_t sld = ptx::sdesc_mnmajor_sw128(slo, 16384, 1024);
+            const uint64_t kd0 = ptx::sdesc_kmajor_sw128(kt), kd1 = ptx::sdesc_kmajor_sw128(kt + 8192);
+            const uint64_t vd = ptx::sdesc_mnmajor_sw128(vt, 8192, 1024);
+            const uint64_t pd = ptx::sdesc_kmajor_sw128(pt);
+            bool ok = ptx::mbar_wait_bounded(s_ready, 0, kTries);
+            for (int m = 0; m < n_mt && ok; ++m) {
+                const int qi = m & 1, ob = m & 1;
+                ok = ptx::mbar_wait_bounded(norm ? &q_ready[qi] : &q_full[qi], (m >> 1) & 1, kTries);
+                if (ok && m >= 2) ok = ptx::mbar_wait_bounded(&o_empty[ob], ((m >> 1) - 1) & 1, kTries);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qb + qi * 32768);
+                const uint64_t qd1 = ptx::sdesc_kmajor_sw128(qb + qi * 32768 + 16384);
+                const uint32_t t_o = tmem + (uint32_t)(ob * 128), t_si = tmem + 256 + (uint32_t)(ob * 64);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                    ptx::umma_f16(t_o, a, shd + (uint64_t)(128 * kk), id_qs, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                    ptx::umma_f16(t_o, a, sld + (uint64_t)(128 * kk), id_qs, 1u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                    const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
+                    ptx::umma_f16(t_si, a, bd, id_qk, kk > 0);
+                }
+                ptx::umma_commit(&q_empty[qi]);
+                ptx::umma_commit(&si_full[ob]);
+                ok = ptx::mbar_wait_bounded(p_full, m & 1, kTries);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    ptx::umma_f16(t_o, pd + 2 * kk, vd + (uint64_t)(128 * kk), id_pv, 1u);
+                ptx::umma_commit(&o_full[ob]);
             }
-            qz[0] += __shfl_xor_sync(0xffffffffu, qz[0], 1);
-            qz[0] += __shfl_xor_sync(0xffffffffu, qz[0], 2);
-            qz[1] += __shfl_xor_sync(0xffffffffu, qz[1], 1);
-            qz[1] += __shfl_xor_sync(0xffffffffu, qz[1], 2);
+            if (!ok) record_error(P.status, kDevTimeout);
+            ptx::umma_commit(mma_all);
+            ptx::mbar_wait_bounded(mma_all, 0, kTries);
         }
-        // inclusive causal mask inside the chunk, row sums for the normaliser
-        float rsum[2] = {0.0f, 0.0f};
-        uint32_t pa[4][4];
+    } else {
+        // ---- warps 2-5: thread = tile row (TMEM lane)
+        const int lb = (warp & 3) * 32, r = lb + lane, et = tid - 64;  // et: 0..127
+        // S_{c-1} (fp32, row = key feature) into bf16 hi + lo, MN-major: row i of
+        // value block jb at jb * 16384 + i * 128, chunk of 8 dims swizzled by i % 8
+        const float* Sp = P.U + (((int64_t)b * P.H_kv + g) * P.nch + c) * kD * kD;
+        for (int rr = warp - 2; rr < kD; rr += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(Sp + (int64_t)rr * kD + lane * 4);
+            const int j = lane * 4, jb = j >> 6, cc = (j & 63) >> 3;
+            const int off = jb * 16384 + rr * 128 + (((cc ^ (rr & 7)) << 4) | ((j & 7) << 1));
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(f.x, f.y), h1 = __floats2bfloat162_rn(f.z, f.w);
+            const float2 g0 = __bfloat1622float2(h0), g1 = __bfloat1622float2(h1);
+            const __nv_bfloat162 l0 = __floats2bfloat162_rn(f.x - g0.x, f.y - g0.y);
+            const __nv_bfloat162 l1 = __floats2bfloat162_rn(f.z - g1.x, f.w - g1.y);
+            *reinterpret_cast<uint2*>(shi + off) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+            *reinterpret_cast<uint2*>(slo + off) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+        }
+        if (norm) zc[et] = P.Z[(((int64_t)b * P.H_kv + g) * P.nch + c) * kD + et];
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 2-5, unconditionally: z is in
+        bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(kv_full, 0, kTries));
+        // phi(K_c) for the intra-chunk scores (rows past T: phi(0) = 1, but
+        // they are masked: a key past T is past every valid query)
+        if (ok && norm) phi_inplace(kt, 16384, et, 128);
+        ptx::fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(s_ready);
+        // elu+1 mode: each thread applies phi to its own row of query tile m in
+        // place and takes phi(q) . z_{c-1} of it at once (the producer reuses
+        // the buffer as soon as the tile's MMAs have read it)
+        float qz_next = 0.0f;
+        auto prep_q = [&](int m) {
+            const int qi = m & 1;
+            const bool w = __all_sync(0xffffffffu,
+                                      ptx::mbar_wait_bounded(&q_full[qi], (m >> 1) & 1, kTries));
+            float acc = 0.0f;
+            if (w) {
+                uint8_t* qrow = qb + qi * 32768 + r * 128;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint4* chunk = reinterpret_cast<uint4*>(qrow + half * 16384 + ((cc ^ (r & 7)) << 4));
+                        uint4 u = *chunk;
+                        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int qi = r0 + gid + 8 * (e >> 1);
-                const int kj = n * 8 + 2 * tq + (e & 1);
-                if (kj > qi) sc[n][e] = 0.0f;
-                rsum[e >> 1] += sc[n][e];
+                        for (int x = 0; x < 4; ++x) {
+                            const float2 f = __bfloat1622float2(h2[x]);
+                            h2[x] = __floats2bfloat162_rn(f.x > 0.0f ? f.x + 1.0f : __expf(f.x),
+                                                          f.y > 0.0f ? f.y + 1.0f : __expf(f.y));
+                            const float2 pf = __bfloat1622float2(h2[x]);
+                            const int f0 = half * 64 + cc * 8 + 2 * x;
+                            acc = fmaf(pf.x, zc[f0], fmaf(pf.y, zc[f0 + 1], acc));
+                        }
+                        *chunk = u;
+                    }
+                }
             }
-            const int kk = n >> 1, hi2 = n & 1;
-            pa[kk][0 + 2 * hi2] = ptx::pack_bf16(sc[n][0], sc[n][1]);
-            pa[kk][1 + 2 * hi2] = ptx::pack_bf16(sc[n][2], sc[n][3]);
-        }
-        // + tril(phi(Q) phi(K)^T) V
-#pragma unroll
-        for (int kk = 0; kk < kC / 16; ++kk) {
-#pragma unroll
-            for (int n = 0; n < 16; n += 2) {
-                uint32_t vr[4];
-                const int key = kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-                const int col = (n + (lane >> 4)) * 8;
-                ptx::ldmatrix_x4_trans(vr, vbase + key * kRow + col * 2);
-                ptx::mma_bf16(o[n], pa[kk], vr[0], vr[1]);
-                ptx::mma_bf16(o[n + 1], pa[kk], vr[2], vr[3]);
+            qz_next = acc;
+            ptx::fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&q_ready[qi]);
+            return w;
+        };
+        if (norm && ok && n_mt > 0) ok = prep_q(0);
+        const int tl = r & 63;              // token of this row within the chunk
+        const bool tok_ok = t0 + tl < P.T;
+        for (int m = 0; m < n_mt && ok; ++m) {
+            const int ob = m & 1;
+            const int hh = r >> 6;          // which head of the pair
+            const bool row_ok = tok_ok && 2 * m + hh < P.group;
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&si_full[ob], (m >> 1) & 1, kTries))) {
+                ok = false;
+                break;
             }
-        }
-        float inv[2] = {1.0f, 1.0f};
-        if (norm) {
+            ptx::tc_fence_after();
+            uint32_t sr[64];
+            ptx::tmem_ld32(tmem + ((uint32_t)lb << 16) + 256 + (uint32_t)(ob * 64), *reinterpret_cast<uint32_t(*)[32]>(sr));
+            ptx::tmem_ld32(tmem + ((uint32_t)lb << 16) + 256 + (uint32_t)(ob * 64 + 32),
+                           *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+            ptx::tmem_ld_wait();
+            // tril: keys j <= this row's token (inclusive), row sum for the normaliser
+            float rsum = 0.0f;
+            uint32_t pk[32];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                rsum[x] += __shfl_xor_sync(0xffffffffu, rsum[x], 1);
-                rsum[x] += __shfl_xor_sync(0xffffffffu, rsum[x], 2);
-                inv[x] = 1.0f / (qz[x] + rsum[x]);
+            for (int j = 0; j < kC; j += 2) {
+                const float a0 = j <= tl ? __uint_as_float(sr[j]) : 0.0f;
+                const float a1 = j + 1 <= tl ? __uint_as_float(sr[j + 1]) : 0.0f;
+                rsum += a0 + a1;
+                pk[j >> 1] = ptx::pack_bf16(a0, a1);
             }
-        }
-        const int hq = g * P.group + h;
+            // the P tile is free once the previous tile's P.V has completed
+            if (m > 0 && !__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&o_full[(m - 1) & 1], ((m - 1) >> 1) & 1, kTries))) {
+                ok = false;
+                break;
+            }
+            uint8_t* prow = pt + r * 128;
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const int t = t0 + r0 + gid + 8 * x;
-            if (t >= P.T) continue;
-            bf16* orow = P.o + (((int64_t)b * P.T + t) * P.H_q + hq) * kD;
+            for (int cc = 0; cc < 8; ++cc)
+                *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+            ptx::fence_proxy_async_shared();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(p_full);
+            const float qz = qz_next;  // phi(q) . z_{c-1} of this row (elu+1)
+            if (norm && m + 1 < n_mt && !prep_q(m + 1)) {
+                ok = false;
+                break;
+            }
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&o_full[ob], (m >> 1) & 1, kTries))) {
+                ok = false;
+                break;
+            }
+            ptx::tc_fence_after();
+            const float inv = norm ? 1.0f / (qz + rsum) : 1.0f;
+            bf16* orow = P.o + (((int64_t)b * P.T + t0 + tl) * P.H_q + g * P.group + 2 * m + hh) * kD;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t ov[32];
+                ptx::tmem_ld32(tmem + ((uint32_t)lb << 16) + (uint32_t)(ob * 128 + c0), ov);
+                ptx::tmem_ld_wait();
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-            for (int n = 0; n < 16; ++n)
-                *reinterpret_cast<__nv_bfloat162*>(orow + n * 8 + 2 * tq) =
-                    __floats2bfloat162_rn(o[n][2 * x] * inv[x], o[n][2 * x + 1] * inv[x]);
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(ptx::pack_bf16(__uint_as_float(ov[8 * e]) * inv, __uint_as_float(ov[8 * e + 1]) * inv),
+                                            ptx::pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv),
+                                            ptx::pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv),
+                                            ptx::pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv));
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&o_empty[ob]);
         }
+        if (!ok && lane == 0) record_error(P.status, kDevTimeout);
     }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -353,7 +534,7 @@ size_t fast_linear_prefill_ws_bytes(const Shape& s) {
 bool fast_linear_prefill_supported(const Shape& s, const void* q, const void* k, const void* v) {
     if (s.dtype != LISA_BF16 || s.d != kD || s.chunk != kC) return false;
     if (s.T < 1 || s.group > 64) return false;
-    return aligned16(q) && aligned16(k) && aligned16(v);
+    return aligned16(q) && aligned16(k) && aligned16(v) && tma_encode_fn() != nullptr;
 }
 
 cudaError_t fast_linear_prefill(const Shape& s, const void* q, const void* k, const void* v,
@@ -366,20 +547,30 @@ cudaError_t fast_linear_prefill(const Shape& s, const void* q, const void* k, co
     char* w8 = (char*)ws + kStatusBytes;
     P.U = (float*)w8;
     P.Z = P.U + (size_t)s.B * s.H_kv * P.nch * kD * kD;
+    P.status = (unsigned*)ws;
+    CUtensorMap tq, tk, tv;
+    memset(&tq, 0, sizeof(tq));
+    memset(&tk, 0, sizeof(tk));
+    memset(&tv, 0, sizeof(tv));
+    const uint64_t qrow = (uint64_t)s.H_q * kD, kvrow = (uint64_t)s.H_kv * kD;
+    if (!make_tmap_bf16_3d(&tq, q, qrow, s.T, s.B, qrow, (uint64_t)s.T * qrow, 64, kC) ||
+        !make_tmap_bf16_3d(&tk, k, kvrow, s.T, s.B, kvrow, (uint64_t)s.T * kvrow, 64, kC) ||
+        !make_tmap_bf16_3d(&tv, v, kvrow, s.T, s.B, kvrow, (uint64_t)s.T * kvrow, 64, kC))
+        return cudaErrorInvalidValue;
     static bool attrs[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attrs[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_la_chunk_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_la_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              OutSmem::total);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attrs[dev] = true;
     }
     const int ctas = s.B * s.H_kv * P.nch;
-    k_la_chunk_sums<<<ctas, 256, 0, st>>>(P);
+    k_la_sums_tc<<<ctas, kSumThreads, 0, st>>>(tk, tv, P);
     const int64_t nstate = (int64_t)s.B * s.H_kv * kD * kD;
     k_la_prefix<<<(unsigned)((nstate + 255) / 256), 256, 0, st>>>(P);
-    k_la_chunk_out<<<ctas, 256, OutSmem::total, st>>>(P);
+    k_la_out_tc<<<ctas, kOutThreads, OutSmem::total, st>>>(tq, tk, tv, P);
     return cudaGetLastError();
 }
 
