@@ -180,19 +180,19 @@ class ClockSampler:
                 "period_ms": self.period_ms, "window": "samples inside the timed region"}
 
 
-def time_blocks(step, steps: int, stream, min_seconds: float, max_blocks: int = 4000):
-    """Runs blocks of `steps` back-to-back steps with a CUDA event at every
-    block boundary (no host synchronisation in between) until about
-    `min_seconds` have passed on the device; returns the device time of each
-    block (ms) and the host times at which the timed region started and
-    ended.  The caller brackets it with a barrier and a synchronise."""
+def time_blocks(run_block, stream, min_seconds: float, max_blocks: int = 4000):
+    """Runs blocks (each `run_block(k)` issues one block of K back-to-back
+    steps) with a CUDA event at every block boundary and no host
+    synchronisation in between, until about `min_seconds` have passed on the
+    device; returns the device time of each block (ms) and the host times at
+    which the timed region started and ended.  The caller brackets it with a
+    barrier and a synchronise."""
     import torch
 
     # size the run from one untimed block
     a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a_.record(stream)
-    for i in range(steps):
-        step(i)
+    run_block(0)
     b_.record(stream)
     torch.cuda.synchronize()
     est = max(a_.elapsed_time(b_), 1e-3)
@@ -202,8 +202,7 @@ def time_blocks(step, steps: int, stream, min_seconds: float, max_blocks: int = 
     t0 = time.time()
     ev[0].record(stream)
     for k in range(blocks):
-        for i in range(steps):
-            step(k * steps + i)
+        run_block(k)
         ev[k + 1].record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
@@ -305,21 +304,29 @@ def run_gpu(args, wl, rank, world, device):
     torch.cuda.synchronize()
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
+
+    def run_block(k):  # noqa: ARG001
+        for i in range(args.steps):
+            step(i)
+
+    graph = None
     if args.graphs:
-        # one CUDA graph per state copy, captured from the same call: a timed
-        # step is one graph launch, so the host's launch cost stays off the GPU
-        for c in copies:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                lisa.lisa_decode_step(D, c["a"], c["ws"])
-            c["graph"] = g
+        # one CUDA graph holding the K steps of a block (cycling through the
+        # state copies): a timed block is one graph launch, so the host's launch
+        # cost stays off the GPU, and each step's kernel is a programmatic
+        # dependent of the one before it (its launch and shared-memory set-up
+        # overlap the previous step's end)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(args.steps):
+                lisa.lisa_decode_step(D, copies[i % len(copies)]["a"], copies[i % len(copies)]["ws"])
         stream = torch.cuda.current_stream()
 
-        def step(i):  # noqa: F811
-            copies[i % len(copies)]["graph"].replay()
+        def run_block(k):  # noqa: F811,ARG001
+            graph.replay()
 
-        for i in range(args.warmup):
-            step(i)
+        for _ in range(max(1, args.warmup // max(1, args.steps)) + 1):
+            run_block(0)
         torch.cuda.synchronize()
         for c in copies:
             assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
@@ -338,12 +345,13 @@ def run_gpu(args, wl, rank, world, device):
     except Exception:
         gpu_id = str(device.index)
     with ClockSampler(gpu_id) as clk:
-        blocks, w0, w1 = time_blocks(step, args.steps, stream, args.min_seconds)
+        blocks, w0, w1 = time_blocks(run_block, stream, args.min_seconds)
     if world > 1:
         dist.barrier()
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], stream) == lisa.LISA_OK
     total_ms = max_over_ranks(statistics.median(blocks), device, world)
+    del graph
 
     # ---- end to end through the public API with host buffers
     pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
@@ -394,8 +402,9 @@ def run_gpu(args, wl, rank, world, device):
                          f"{args.rotate} x {bytes_['total'] / 1e6:.1f} MB touched per cycle",
                    "step": "decode step: append, linear update+readout, indexer scan, "
                            "top-M, sparse attention, gate (one cooperative kernel)",
-                   "launch": "CUDA graph replay of lisa_decode_step" if args.graphs
-                             else "lisa_decode_step from the host"},
+                   "launch": "one CUDA graph of the K lisa_decode_step calls of a block, "
+                             "each kernel a programmatic dependent of the previous one"
+                             if args.graphs else "lisa_decode_step from the host"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "frac_of_8TBs": achieved / 8000.0,
@@ -420,33 +429,34 @@ def run_gpu(args, wl, rank, world, device):
 
 # ----------------------------------------------------------------------------- helpers
 def graph_timed(calls, steps: int, warmup: int):
-    """Captures one CUDA graph per call (each a closure issuing one library call
-    on the current stream) and replays them in rotation: `warmup` untimed
-    replays, then `steps` between one event pair on the launching stream.
-    Returns the device time per replay in ms."""
+    """Captures one CUDA graph issuing every call once (each a closure issuing
+    one library call on the current stream, typically one per state copy) and
+    replays it: enough untimed replays for `warmup` calls, then enough for at
+    least `steps` calls between one event pair on the launching stream.
+    Returns the device time per call in ms."""
     import torch
 
     for c in calls:
         c()
     torch.cuda.synchronize()
-    graphs = []
-    for c in calls:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
             c()
-        graphs.append(g)
     cur = torch.cuda.current_stream()
-    for i in range(warmup):
-        graphs[i % len(graphs)].replay()
+    per = len(calls)
+    for _ in range(max(1, math.ceil(warmup / per))):
+        g.replay()
     torch.cuda.synchronize()
+    reps = max(1, math.ceil(steps / per))
     a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a_.record(cur)
-    for i in range(steps):
-        graphs[i % len(graphs)].replay()
+    for _ in range(reps):
+        g.replay()
     b_.record(cur)
     torch.cuda.synchronize()
-    ms = a_.elapsed_time(b_) / steps
-    del graphs
+    ms = a_.elapsed_time(b_) / (reps * per)
+    del g
     return ms
 
 
@@ -621,29 +631,12 @@ def run_next_rows(args, wl, copies, D, stream):
 
     hbm_peak, _, peak_kind = _peaks()
     out = {}
-    # ---- sliding-window decode step (no indexer), graphs as for the main line
-    for c in copies:
-        lisa.lisa_decode_step_window(D, c["a"], c["ws"], stream)
-    torch.cuda.synchronize()
-    graphs = []
-    for c in copies:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            lisa.lisa_decode_step_window(D, c["a"], c["ws"])
-        graphs.append(g)
+    # ---- sliding-window decode step (no indexer), one graph over the copies
     cur = torch.cuda.current_stream()
-    for i in range(args.warmup):
-        graphs[i % len(graphs)].replay()
-    torch.cuda.synchronize()
-    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_.record(cur)
-    for i in range(args.steps):
-        graphs[i % len(graphs)].replay()
-    b_.record(cur)
-    torch.cuda.synchronize()
+    ms = graph_timed([lambda c=c: lisa.lisa_decode_step_window(D, c["a"], c["ws"]) for c in copies],
+                     args.steps, args.warmup)
     for c in copies:
         assert lisa.lisa_check_status(c["ws"], cur) == lisa.LISA_OK
-    ms = a_.elapsed_time(b_) / args.steps
     wb = window_bytes(wl)
     out["window"] = {
         "what": "decode step with the Stage-1 sliding window (last M positions, no indexer): "
@@ -695,26 +688,10 @@ def run_next_rows(args, wl, copies, D, stream):
                               dv["q"], dv["k_new"], dv["v_new"], dv["gate"], c["kc"], c["vc"], kc8,
                               c["S"], None, c["o"])
         pf.append(dict(a=a8, ws=lisa.workspace(D8, lisa.LISA_OP_DECODE_STEP, stream.device)))
-    for c in pf:
-        lisa.lisa_decode_step(D8, c["a"], c["ws"], stream)
-    torch.cuda.synchronize()
-    for c in pf:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            lisa.lisa_decode_step(D8, c["a"], c["ws"])
-        c["graph"] = g
-    for i in range(args.warmup):
-        pf[i % len(pf)]["graph"].replay()
-    torch.cuda.synchronize()
-    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_.record(cur)
-    for i in range(args.steps):
-        pf[i % len(pf)]["graph"].replay()
-    b_.record(cur)
-    torch.cuda.synchronize()
+    ms = graph_timed([lambda c=c: lisa.lisa_decode_step(D8, c["a"], c["ws"]) for c in pf],
+                     args.steps, args.warmup)
     for c in pf:
         assert lisa.lisa_check_status(c["ws"], cur) == lisa.LISA_OK
-    ms = a_.elapsed_time(b_) / args.steps
     pb = decode_bytes(wl8)
     out["paper_form"] = {
         "what": "decode step with the paper's indexer form: a key per indexer head "

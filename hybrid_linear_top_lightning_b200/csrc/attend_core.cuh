@@ -190,7 +190,7 @@ __device__ __forceinline__ void attn_stage16(const uint32_t (&qf)[8][2], uint32_
         mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
         mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
         const float m_new = fmaxf(m[h], mt);
-        corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m[h] - m_new);
+        corr[h] = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m[h] - m_new);
         m[h] = m_new;
         l[h] *= corr[h];
     }
@@ -198,7 +198,7 @@ __device__ __forceinline__ void attn_stage16(const uint32_t (&qf)[8][2], uint32_
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const float mm = m[e & 1];
-        pr[e] = (mm == -INFINITY) ? 0.0f : exp2f(v[e] - mm);
+        pr[e] = (mm == -INFINITY) ? 0.0f : ptx::ex2(v[e] - mm);
         l[e & 1] += pr[e];
     }
 #pragma unroll
@@ -315,7 +315,7 @@ __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spo
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
             const float m_new = fmaxf(m[h], mt);
-            corr[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m[h] - m_new);
+            corr[h] = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m[h] - m_new);
             m[h] = m_new;
             l[h] *= corr[h];
         }
@@ -323,7 +323,7 @@ __device__ __forceinline__ void attn_core(const AttQ& q, uint8_t* ring, int* spo
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float mm = m[e & 1];
-            p[e] = (mm == -INFINITY) ? 0.0f : exp2f(v[e] - mm);
+            p[e] = (mm == -INFINITY) ? 0.0f : ptx::ex2(v[e] - mm);
             l[e & 1] += p[e];
         }
 #pragma unroll

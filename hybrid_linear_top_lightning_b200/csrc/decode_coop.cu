@@ -390,7 +390,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // its arrival at exchange 1, word 3 = the poll limit of that exchange (0:
     // the default).  Tests use it to watch a bounded wait give up.
     uint2 hook = make_uint2(0u, 0u);
-    if (tid == 0) hook = __ldcg(reinterpret_cast<const uint2*>(P.status + 2));
 
     for (int i = tid; i < 4096; i += kThreads) shist[i] = 0u;
     if (tid == 0) {
@@ -404,6 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    // Launched as a programmatic dependent of the previous kernel on the stream,
+    // this CTA has set up its shared memory while that kernel finished; nothing
+    // global is touched before the previous kernel has completed.  The next
+    // kernel may start its own set-up once every CTA of this one is resident.
+    ptx::pdl_wait_prior();
+    ptx::pdl_launch_dependents();
+    if (tid == 0) hook = __ldcg(reinterpret_cast<const uint2*>(P.status + 2));
 
     // ======================================================== A: scan | linear branch
     if (warp < kSlots) {
@@ -908,35 +914,85 @@ __global__ void __launch_bounds__(kThreads, 1)
         find_bin<NT>(shist, 1024, need1, rmisc, rt, kRefBar);
         const uint32_t D2 = (uint32_t)rmisc[0];
         const int need2 = rmisc[1];
+        const int cnt2 = rmisc[2];  // keys of the sequence in the 20-bit bin (D1, D2)
         gsync<NT>(kRefBar);
-        // third digit: key bits [9:0] of the candidates that share D2
-        for (int i = rt; i < 1024; i += NT) shist[i] = 0u;
-        gsync<NT>(kRefBar);
-        for (int i = rt; i < C; i += NT) {
-            const uint32_t key = cand_at(i).x;
-            if (((key >> 10) & 1023u) == D2) atomicAdd(shist + (key & 1023u), 1u);
-        }
-        gsync<NT>(kRefBar);
-        find_bin<NT>(shist, 1024, need2, rmisc, rt, kRefBar);
-        const uint32_t tau = (D1 << 20) | (D2 << 10) | (uint32_t)rmisc[0];
-        const int need_eq = rmisc[1];
-        const bool all_ties = need_eq >= rmisc[2];
-        gsync<NT>(kRefBar);
-        int tie_prefix = 0;
-        if (!all_ties) {
-            // keys equal to tau at positions before this CTA's range
-            if (rt == 0) rmisc[3] = 0;
+        uint32_t tau;
+        int need_eq, tie_prefix = 0;
+        bool all_ties;
+        if (cnt2 <= 32) {
+            // few keys share the 20-bit bin (the usual case): collect them and
+            // let one warp rank them directly (descending key; every key equal
+            // to tau is among them, so the ties before this CTA's range are too)
+            uint2* few = reinterpret_cast<uint2*>(shist);
+            if (rt == 0) rmisc[4] = 0;
             gsync<NT>(kRefBar);
-            int c = 0;
             for (int i = rt; i < C; i += NT) {
                 const uint2 e = cand_at(i);
-                c += (e.x == tau && (int)e.y < k0) ? 1 : 0;
+                if (((e.x >> 10) & 1023u) == D2) {
+                    const int at = atomicAdd(rmisc + 4, 1);
+                    if (at < 32) few[at] = e;
+                }
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-            if (lane == 0 && c) atomicAdd(rmisc + 3, c);
             gsync<NT>(kRefBar);
-            tie_prefix = rmisc[3];
+            if (rt < 32) {
+                const int m = min(rmisc[4], 32);
+                const uint2 me = rt < m ? few[rt] : make_uint2(0u, 0u);
+                int gt = 0, eq = 0;
+                for (int o = 0; o < m; ++o) {
+                    const uint32_t kx = __shfl_sync(0xffffffffu, me.x, o);
+                    gt += kx > me.x ? 1 : 0;
+                    eq += kx == me.x ? 1 : 0;
+                }
+                const bool hit = rt < m && gt < need2 && need2 <= gt + eq;
+                const unsigned who = __ballot_sync(0xffffffffu, hit);
+                const int src = who ? __ffs(who) - 1 : 0;
+                const uint32_t tk = __shfl_sync(0xffffffffu, me.x, src);
+                const int tgt = __shfl_sync(0xffffffffu, gt, src);
+                const int teq = __shfl_sync(0xffffffffu, eq, src);
+                const unsigned before =
+                    __ballot_sync(0xffffffffu, rt < m && me.x == tk && (int)me.y < k0);
+                if (rt == 0) {
+                    rmisc[0] = who ? (int)(tk & 1023u) : 0;  // (safe values if the counts disagree)
+                    rmisc[1] = who ? need2 - tgt : 1;
+                    rmisc[2] = who ? teq : 0;
+                    rmisc[3] = __popc(before);
+                }
+            }
+            gsync<NT>(kRefBar);
+            tau = (D1 << 20) | (D2 << 10) | (uint32_t)rmisc[0];
+            need_eq = rmisc[1];
+            all_ties = need_eq >= rmisc[2];
+            if (!all_ties) tie_prefix = rmisc[3];
+            gsync<NT>(kRefBar);
+        } else {
+            // third digit: key bits [9:0] of the candidates that share D2
+            for (int i = rt; i < 1024; i += NT) shist[i] = 0u;
+            gsync<NT>(kRefBar);
+            for (int i = rt; i < C; i += NT) {
+                const uint32_t key = cand_at(i).x;
+                if (((key >> 10) & 1023u) == D2) atomicAdd(shist + (key & 1023u), 1u);
+            }
+            gsync<NT>(kRefBar);
+            find_bin<NT>(shist, 1024, need2, rmisc, rt, kRefBar);
+            tau = (D1 << 20) | (D2 << 10) | (uint32_t)rmisc[0];
+            need_eq = rmisc[1];
+            all_ties = need_eq >= rmisc[2];
+            gsync<NT>(kRefBar);
+            if (!all_ties) {
+                // keys equal to tau at positions before this CTA's range
+                if (rt == 0) rmisc[3] = 0;
+                gsync<NT>(kRefBar);
+                int c = 0;
+                for (int i = rt; i < C; i += NT) {
+                    const uint2 e = cand_at(i);
+                    c += (e.x == tau && (int)e.y < k0) ? 1 : 0;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+                if (lane == 0 && c) atomicAdd(rmisc + 3, c);
+                gsync<NT>(kRefBar);
+                tie_prefix = rmisc[3];
+            }
         }
         // this CTA's selected keys of digit D1, appended after the certain ones
         // (ties ranked by position)
@@ -1223,16 +1279,28 @@ cudaError_t coop_decode_step(const Shape& s, const lisa_decode_args& a, void* ws
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the exchanges wait on peers
     attr[0].val.cooperative = 1;
+    // a programmatic dependent of the previous kernel on the stream: its launch
+    // and shared-memory set-up overlap that kernel's end (the kernel waits for
+    // it to complete before touching global memory)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(s.B * pl.ncta);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_coop, tmap_slot, tmap_tail, P);
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_decode_coop, tmap_slot, tmap_tail, P);
+    if (e == cudaErrorInvalidValue || e == cudaErrorNotSupported) {
+        // a driver that takes no programmatic dependency with a cooperative grid
+        (void)cudaGetLastError();
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k_decode_coop, tmap_slot, tmap_tail, P);
+    }
+    return e;
 }
 
 }  // namespace lisa

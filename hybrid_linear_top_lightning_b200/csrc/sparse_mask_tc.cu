@@ -22,9 +22,10 @@
 //                    MN-major straight from its TMA tile) into the TMEM
 //                    output; warps 2-5 (one query row per thread, the row's
 //                    TMEM lane) read S, keep only the selected keys, update
-//                    the row's running max and sum (the output is rescaled in
-//                    TMEM only when the max grows by more than 2^8, which
-//                    leaves the result exact), write P as bf16 into shared
+//                    the row's running reference and sum (the output is
+//                    rescaled in TMEM only when a selected score exceeds the
+//                    reference by more than 2^64, which leaves the result
+//                    exact), write P as bf16 into shared
 //                    memory in the MMA's swizzled layout, and at the end
 //                    normalise O and store it.
 //
@@ -52,11 +53,13 @@ constexpr int kQT = 128;          // query rows per tile (MMA M)
 constexpr int kKT = 64;           // keys per tile
 constexpr int kD = 128;           // head dimension of this path
 constexpr int kStages = 4;        // K (and V) tiles in flight
-constexpr int kThreads = 192;     // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kThreads = 320;     // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 softmax (two groups)
 constexpr int kMaxTiles = 2048;   // key tiles one query tile may visit (keys <= 131072)
 constexpr uint32_t kTries = 1u << 22;
-constexpr float kLazy = 8.0f;     // rescale the output when the max grows by more (log2)
-constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128
+constexpr float kLazy = 64.0f;    // move the softmax reference when a score exceeds it by more (log2)
+constexpr uint32_t kTmemCols = 512;  // 4 score buffers at columns 0-255, the groups' outputs at 256, 384
+constexpr int kSBuf = 4;             // score buffers: tile i uses i % 4 (group i % 2 owns two)
+constexpr uint32_t kOCol = kSBuf * kKT;
 
 struct MaskParams {
     int T, n_past, M, Lw, nqt, nkw;
@@ -118,11 +121,12 @@ struct Smem {
     static constexpr int q = 0;                                  // 2 boxes of 64 dims x 128 rows
     static constexpr int k = q + 2 * 16384;                      // kStages x (2 x 64 dims x 64 keys)
     static constexpr int v = k + kStages * 16384;                // the same for V
-    static constexpr int p = v + kStages * 16384;                // 128 rows x 64 keys bf16
-    static constexpr int list = p + 16384;                       // int[kMaxTiles]
+    static constexpr int p = v + kStages * 16384;                // 2 groups x 128 rows x 64 keys bf16
+    static constexpr int list = p + 2 * 16384;                   // int[kMaxTiles]
     static constexpr int bars = list + kMaxTiles * 4;            // mbarriers
     static constexpr int misc = bars + 32 * 8;                   // tmem base, tile count, fail
-    static constexpr int total = misc + 64 + 1024;               // + base alignment slack
+    static constexpr int xch = misc + 64;                        // group 1's max and sum per row
+    static constexpr int total = xch + 2 * kQT * 4 + 1024;       // + base alignment slack
 };
 static_assert(Smem::total <= 227 * 1024, "shared memory per CTA");
 
@@ -147,11 +151,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* k_empty = k_full + kStages;
     uint64_t* v_full = k_empty + kStages;
     uint64_t* v_empty = v_full + kStages;
-    uint64_t* s_full = v_empty + kStages;   // [2]
-    uint64_t* s_empty = s_full + 2;         // [2]
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* pv_done = p_full + 1;
-    uint64_t* mma_all = pv_done + 1;        // every MMA this CTA issued has completed
+    uint64_t* s_full = v_empty + kStages;   // [4] score buffer i % 4 written
+    uint64_t* s_empty = s_full + kSBuf;     // [4] and read by its softmax group
+    uint64_t* p_full = s_empty + kSBuf;     // [2] group's P tile written
+    uint64_t* pv_done = p_full + 2;         // [2] group's P.V product done
+    uint64_t* mma_all = pv_done + 2;        // every MMA this CTA issued has completed
+    float* xm = reinterpret_cast<float*>(base + Smem::xch);
+    float* xl = xm + kQT;
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + Smem::misc);  // [0] tmem, [1] tiles, [2] fail
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -171,12 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&v_full[s], 1);
             ptx::mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kSBuf; ++s) {
             ptx::mbar_init(&s_full[s], 1);
             ptx::mbar_init(&s_empty[s], 4);
         }
-        ptx::mbar_init(p_full, 4);
-        ptx::mbar_init(pv_done, 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&p_full[s], 4);
+            ptx::mbar_init(&pv_done[s], 1);
+        }
         ptx::mbar_init(mma_all, 1);
         ptx::fence_mbar_init();
         misc[2] = 0u;
@@ -215,7 +223,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = misc[0];
     const int n = (int)misc[1];
-    const uint32_t t_o = tmem + 128;  // output columns
 
     if (warp == 0) {
         if (lane == 0 && n > 0) {
@@ -256,16 +263,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && n > 0) {
-            // ---- MMA issuer
+            // ---- MMA issuer: S_i into score buffer i % 2; P_i V_i into the
+            // output of softmax group i % 2
             const uint32_t idesc_s = ptx::idesc_bf16_f32(kQT, kKT);
             const uint32_t idesc_pv = ptx::idesc_bf16_f32_bmn(kQT, kD);
             const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs), qd1 = ptx::sdesc_kmajor_sw128(qs + 16384);
-            const uint64_t pd = ptx::sdesc_kmajor_sw128(ps);
             bool ok = wait_bar(q_full, 0);
             auto issue_s = [&](int i) {
-                const int s = i % kStages, sb = i & 1;
+                const int s = i % kStages, sb = i % kSBuf;
                 ok = ok && wait_bar(&k_full[s], (i / kStages) & 1);
-                if (ok && i >= 2) ok = wait_bar(&s_empty[sb], ((i >> 1) - 1) & 1);
+                if (ok && i >= kSBuf) ok = wait_bar(&s_empty[sb], ((i / kSBuf) - 1) & 1);
                 if (!ok) return;
                 ptx::tc_fence_after();
                 const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
@@ -279,21 +286,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::umma_commit(&k_empty[s]);
                 ptx::umma_commit(&s_full[sb]);
             };
-            issue_s(0);
+            // the score products run two tiles ahead of the P.V products, so a
+            // softmax group finds its next tile's scores ready when it finishes one
+            int next_s = 0;
             for (int i = 0; i < n && ok; ++i) {
-                if (i + 1 < n) issue_s(i + 1);
-                const int s = i % kStages;
-                ok = ok && wait_bar(p_full, i & 1);
+                while (ok && next_s < n && next_s <= i + 2) issue_s(next_s++);
+                const int s = i % kStages, grp = i & 1;
+                ok = ok && wait_bar(&p_full[grp], (i >> 1) & 1);
                 ok = ok && wait_bar(&v_full[s], (i / kStages) & 1);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                const uint64_t pd = ptx::sdesc_kmajor_sw128(ps + grp * 16384);
                 const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk)
-                    ptx::umma_f16(t_o, pd + 2 * kk, vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
-                                  (i > 0 || kk > 0) ? 1u : 0u);
+                    ptx::umma_f16(tmem + kOCol + (uint32_t)(grp * kD), pd + 2 * kk,
+                                  vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
+                                  (i >= 2 || kk > 0) ? 1u : 0u);
                 ptx::umma_commit(&v_empty[s]);
-                ptx::umma_commit(pv_done);
+                ptx::umma_commit(&pv_done[grp]);
             }
             if (!ok) {
                 misc[2] = 1u;
@@ -304,131 +315,164 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_wait_bounded(mma_all, 0, kTries);
         }
     } else {
-        // ---- softmax: thread = query row (its TMEM lane)
+        // ---- softmax: two groups of four warps take alternate key tiles
+        // (group grp: tiles grp, grp + 2, ...), each with its own running max
+        // and sum per row and its own output in TMEM; thread = query row
+        const int grp = (warp - 2) >> 2;
         const int lb = (warp & 3) * 32;
         const int r = lb + lane;
         const int t = q0 + r;
         const bool valid = t < P.T;
         const uint32_t* mrow = P.mask + ((int64_t)b * P.T + (valid ? t : 0)) * P.Lw;
         const uint32_t t_row = tmem + ((uint32_t)lb << 16);
+        const uint32_t t_out = t_row + kOCol + (uint32_t)(grp * kD);  // and output
+        uint8_t* prow = ps + grp * 16384 + r * 128;
+        const int mine = grp < n ? (n - grp + 1) / 2 : 0;  // tiles of this group
         float m_used = -INFINITY, l = 0.0f;
-        uint2 mk_next = make_uint2(0u, 0u);
-        if (valid && n > 0) mk_next = __ldg(reinterpret_cast<const uint2*>(mrow) + list[0]);
-        int pv_waited = 0;  // PV products known complete
+        // the row's mask words of this group's next two tiles
+        uint2 mk_a = make_uint2(0u, 0u), mk_b = make_uint2(0u, 0u);
+        if (valid && mine > 0) mk_a = __ldg(reinterpret_cast<const uint2*>(mrow) + list[grp]);
+        if (valid && mine > 1) mk_b = __ldg(reinterpret_cast<const uint2*>(mrow) + list[grp + 2]);
         bool ok = true;
-        for (int i = 0; i < n; ++i) {
-            const int sb = i & 1;
-            const uint2 mk = mk_next;
-            if (valid && i + 1 < n) mk_next = __ldg(reinterpret_cast<const uint2*>(mrow) + list[i + 1]);
+        for (int j = 0; j < mine; ++j) {
+            const int i = 2 * j + grp;
+            const uint2 mk = mk_a;
+            mk_a = mk_b;
+            if (valid && j + 2 < mine) mk_b = __ldg(reinterpret_cast<const uint2*>(mrow) + list[i + 4]);
+            const int sb = i % kSBuf;
+            const uint32_t t_s = t_row + (uint32_t)(sb * kKT);  // this tile's score buffer
             // (waits agree across the warp: the TMEM accesses that follow are collective)
-            if (!__all_sync(0xffffffffu, wait_bar(&s_full[sb], (i >> 1) & 1))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&s_full[sb], (i / kSBuf) & 1))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
+            // the tile's 64 scores, both loads in flight before the one wait;
+            // the score buffer is then free for the MMA to refill
             uint32_t sr[64];
-            ptx::tmem_ld32(t_row + (uint32_t)(sb * kKT), *reinterpret_cast<uint32_t(*)[32]>(sr));
-            ptx::tmem_ld32(t_row + (uint32_t)(sb * kKT + 32), *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+            ptx::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
+            ptx::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
             ptx::tmem_ld_wait();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
-            // the tile's largest selected score (the scale is positive)
-            float mx = -INFINITY;
+            // The reference m_used only has to keep every selected p = 2^(s - m_used)
+            // far from overflow: the largest score of the whole tile (selected or
+            // not, four chains) bounds the selected ones, so the masked maximum is
+            // taken only when that bound could move the reference: for the row's
+            // first selected keys, or when it exceeds the reference by 2^kLazy.
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int k = 0; k < 64; ++k) {
-                const uint32_t w = k < 32 ? mk.x : mk.y;
-                if ((w >> (k & 31)) & 1u) mx = fmaxf(mx, __uint_as_float(sr[k]));
+            for (int k = 0; k < 64; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sr[k]));
+            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
+            const bool any_sel = (mk.x | mk.y) != 0u;
+            if (any_sel && (m_used == -INFINITY || mx > m_used + kLazy)) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 64; ++k) {
+                    const uint32_t w = k < 32 ? mk.x : mk.y;
+                    if (w & (1u << (k & 31))) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sr[k]));
+                }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
+            } else {
+                mx = -INFINITY;  // the reference stays
             }
-            mx = mx == -INFINITY ? -INFINITY : mx * P.scale_log2;
             // the running max moves when a selected score exceeds it by more
-            // than 2^kLazy (the output and sum are rescaled then), or when the
-            // row meets its first selected key (the output is still zero)
+            // than 2^kLazy (the output and sum are rescaled by alpha then), or
+            // when the row meets its first selected key (its output is still zero)
             const bool first = m_used == -INFINITY && mx != -INFINITY;
             const bool grow = m_used != -INFINITY && mx > m_used + kLazy;
-            if (__any_sync(0xffffffffu, grow)) {
-                // the output must hold every product so far before it is rescaled
-                if (i > 0 && pv_waited < i) {
-                    if (!__all_sync(0xffffffffu, wait_bar(pv_done, (i - 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                    pv_waited = i;
-                }
-                ptx::tc_fence_after();
-                const float alpha = grow ? exp2f(m_used - mx) : 1.0f;
-#pragma unroll 1
-                for (int c = 0; c < kD; c += 32) {
-                    uint32_t ov[32];
-                    ptx::tmem_ld32(t_row + 128 + (uint32_t)c, ov);
-                    ptx::tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                    ptx::tmem_st32(t_row + 128 + (uint32_t)c, ov);
-                }
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
-                l *= alpha;
-            }
+            const float alpha = grow ? exp2f(m_used - mx) : 1.0f;
             if (first || grow) m_used = mx;
             // probabilities of the selected keys (bf16 pairs), zero elsewhere
             uint32_t pk[32];
-            float lsum = 0.0f;
+            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int k = 0; k < 64; k += 2) {
                 const uint32_t w = k < 32 ? mk.x : mk.y;
-                const bool s0 = (w >> (k & 31)) & 1u, s1 = (w >> ((k + 1) & 31)) & 1u;
-                const float p0 = s0 ? exp2f(fmaf(__uint_as_float(sr[k]), P.scale_log2, -m_used)) : 0.0f;
-                const float p1 = s1 ? exp2f(fmaf(__uint_as_float(sr[k + 1]), P.scale_log2, -m_used)) : 0.0f;
-                lsum += p0 + p1;
+                const bool s0 = (w & (1u << (k & 31))) != 0u, s1 = (w & (1u << ((k + 1) & 31))) != 0u;
+                const float p0 = s0 ? ptx::ex2(fmaf(__uint_as_float(sr[k]), P.scale_log2, -m_used)) : 0.0f;
+                const float p1 = s1 ? ptx::ex2(fmaf(__uint_as_float(sr[k + 1]), P.scale_log2, -m_used)) : 0.0f;
+                l4[(k >> 1) & 3] += p0 + p1;
                 pk[k >> 1] = ptx::pack_bf16(p0, p1);
             }
-            l += lsum;
-            // the P tile is free once the previous product has read it
-            if (i > 0 && pv_waited < i) {
-                if (!__all_sync(0xffffffffu, wait_bar(pv_done, (i - 1) & 1))) {
-                    ok = false;
-                    break;
-                }
-                pv_waited = i;
+            l = l * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
+            // this group's previous product has completed: its P tile is free
+            // and its output holds every product so far
+            if (j > 0 && !__all_sync(0xffffffffu, wait_bar(&pv_done[grp], (j - 1) & 1))) {
+                ok = false;
+                break;
             }
             // row r of P: 128 bytes, 16-byte chunk c at chunk c ^ (r % 8)
-            uint8_t* prow = ps + r * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            if (__any_sync(0xffffffffu, grow)) {
+                ptx::tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < kD; c += 16) {
+                    uint32_t ov[16];
+                    ptx::tmem_ld16(t_out + (uint32_t)c, ov);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    ptx::tmem_st16(t_out + (uint32_t)c, ov);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+            }
             ptx::fence_proxy_async_shared();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(p_full);
+            if (lane == 0) ptx::mbar_arrive(&p_full[grp]);
         }
         if (!ok) {
             misc[2] = 1u;
             if (lane == 0) record_error(P.status, kDevTimeout);
         }
-        // ---- epilogue: O / l, bf16, to global memory
-        bf16* orow = P.o + (((int64_t)b * P.T + (valid ? t : 0)) * P.H_q + h) * kD;
-        const bool have = __all_sync(0xffffffffu, ok && n > 0 && wait_bar(pv_done, (n - 1) & 1));
-        if (have) ptx::tc_fence_after();
-        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+        // ---- epilogue: group 1 hands its (max, sum) over; group 0 merges the
+        // two outputs, divides by the sum and stores bf16
+        const bool have = __all_sync(0xffffffffu,
+                                     ok && (mine == 0 || wait_bar(&pv_done[grp], (mine - 1) & 1)));
+        if (grp == 1) {
+            xm[r] = have ? m_used : -INFINITY;
+            xl[r] = have ? l : 0.0f;
+        }
+        ptx::tc_fence_before();
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // both groups, unconditionally
+        ptx::tc_fence_after();
+        if (grp == 0) {
+            const float mb = xm[r], lb2 = xl[r];
+            const float ma = have ? m_used : -INFINITY;
+            const float mm = fmaxf(ma, mb);
+            const float ca = ma == -INFINITY ? 0.0f : exp2f(ma - mm);
+            const float cb = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
+            const float lt = (have ? l : 0.0f) * ca + lb2 * cb;
+            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+            const float wa = ca * inv, wb = cb * inv;
+            bf16* orow = P.o + (((int64_t)b * P.T + (valid ? t : 0)) * P.H_q + h) * kD;
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 32) {
-            uint32_t ov[32];
-            if (have) {
-                ptx::tmem_ld32(t_row + 128 + (uint32_t)c, ov);
+            for (int c = 0; c < kD; c += 16) {
+                uint32_t oa[16], ob[16];
+                ptx::tmem_ld16(t_row + kOCol + (uint32_t)c, oa);
+                ptx::tmem_ld16(t_row + kOCol + kD + (uint32_t)c, ob);
                 ptx::tmem_ld_wait();
-            }
-            uint32_t pkd[16];
+                uint32_t pkd[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                pkd[e] = have ? ptx::pack_bf16(__uint_as_float(ov[2 * e]) * inv,
-                                               __uint_as_float(ov[2 * e + 1]) * inv)
-                              : 0u;
-            if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + c);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    dst[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+                for (int e = 0; e < 8; ++e) {
+                    // an output no product has written is never read (its weight is 0)
+                    const float a0 = wa != 0.0f ? __uint_as_float(oa[2 * e]) * wa : 0.0f;
+                    const float a1 = wa != 0.0f ? __uint_as_float(oa[2 * e + 1]) * wa : 0.0f;
+                    const float b0 = wb != 0.0f ? __uint_as_float(ob[2 * e]) * wb : 0.0f;
+                    const float b1 = wb != 0.0f ? __uint_as_float(ob[2 * e + 1]) * wb : 0.0f;
+                    pkd[e] = ptx::pack_bf16(a0 + b0, a1 + b1);
+                }
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
+                    dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+                    dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+                }
             }
         }
     }

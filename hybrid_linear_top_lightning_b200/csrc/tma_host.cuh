@@ -61,16 +61,17 @@ inline bool make_tmap_bf16_box(CUtensorMap* m, const void* base, uint64_t inner,
 
 // A 3-D bf16 tensor [batch][rows][inner] whose rows are `row_stride` elements
 // apart and whose batches are `batch_stride` elements apart, read in boxes of
-// box_inner (64: 128 bytes) x box_rows x 1 with the 128-byte swizzle.  Rows at
-// or past `rows` read as zero.
+// box_inner (64: 128 bytes) x box_rows x box_batch with the 128-byte swizzle
+// (in shared memory: box_rows x box_batch rows of 128 bytes, rows fastest).
+// Elements past a dimension's end read as zero.
 inline bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                               uint64_t batch, uint64_t row_stride, uint64_t batch_stride,
-                              uint32_t box_inner, uint32_t box_rows) {
+                              uint32_t box_inner, uint32_t box_rows, uint32_t box_batch = 1) {
     EncodeTiledFn fn = tma_encode_fn();
     if (!fn) return false;
     const cuuint64_t gdim[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)batch};
     const cuuint64_t gstride[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)batch_stride * 2};
-    const cuuint32_t box[3] = {box_inner, box_rows, 1};
+    const cuuint32_t box[3] = {box_inner, box_rows, box_batch};
     const cuuint32_t estride[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box,
               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -1,8 +1,9 @@
 """GPU parity of the paper's own indexer form against the oracle: every indexer
 head has its own keys and the head scores are summed without weights
-(LISA, arXiv 2607.19358v1, Sec. 3.2: H_Ik = H_I, w = 1).  The specialised
-kernels take one shared key head; this form runs on the generic kernels,
-through lisa_topm (prefill rows) and lisa_decode_step (bf16 and fp32).
+(LISA, arXiv 2607.19358v1, Sec. 3.2: H_Ik = H_I, w = 1), through lisa_topm
+(prefill rows: the tcgen05 per-head score kernel at 8 indexer heads of 64
+dims in bf16, the generic kernels otherwise) and lisa_decode_step (bf16 and
+fp32).
 """
 import numpy as np
 import pytest
@@ -41,6 +42,31 @@ def test_paper_form_topm_prefill_rows(dtype):
     assert lisa.lisa_check_status(ws) == lisa.LISA_OK
     Dr = ref.Dims(B=wl.B, T=T, n_past=0, N_max=T, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d, H_I=wl.H_I,
                   H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
+    sc = ref.index_scores(Dr, q_I, k_I, w, wl.H_I)
+    r_idx, r_cnt = ref.topm(Dr, sc)
+    g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    for b in range(wl.B):
+        check_topm(g_idx[b], g_cnt[b], r_idx[b], r_cnt[b], sc[b])
+
+
+@pytest.mark.parametrize("n_past,unit_w", [(0, True), (0, False), (300, True)])
+def test_paper_form_topm_prefill_tensor_cores(n_past, unit_w):
+    """8 indexer heads with a key each, bf16: the per-head tcgen05 score GEMM;
+    partial query and key tiles, a call continuing after cached tokens."""
+    wl = inputs.PREFILL_7B.with_(B=2, n=n_past + 700, H_Ik=8, M=160)
+    gen = inputs.Generator(wl)
+    T, L = 700, n_past + 700
+    q_I, k_I = gen.batch("q_I", n_past, L), gen.batch("k_I", 0, L)
+    w = np.ones((wl.B, T, wl.H_I), np.float32) if unit_w else gen.batch("w", n_past, L)
+    D = lisa.make_dims(wl.B, T, n_past, L, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M)
+    idx = torch.empty(wl.B, T, wl.M, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(wl.B, T, dtype=torch.int32, device="cuda")
+    ws = lisa.workspace(D, lisa.LISA_OP_TOPM)
+    lisa.lisa_topm(D, _dv(q_I, torch.bfloat16), _dv(k_I, torch.bfloat16), _dv(w, torch.float32),
+                   wl.H_I, idx, cnt, ws)
+    assert lisa.lisa_check_status(ws) == lisa.LISA_OK
+    Dr = ref.Dims(B=wl.B, T=T, n_past=n_past, N_max=L, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d,
+                  H_I=wl.H_I, H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
     sc = ref.index_scores(Dr, q_I, k_I, w, wl.H_I)
     r_idx, r_cnt = ref.topm(Dr, sc)
     g_idx, g_cnt = idx.cpu().numpy(), cnt.cpu().numpy()
