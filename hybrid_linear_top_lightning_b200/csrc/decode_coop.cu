@@ -873,9 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the first 8 * NT list entries are loaded with the count (entries past it
         // are discarded), the rest, if any, once the count is known
-        uint2 v[8];
+        constexpr int kCL = 16;  // list entries loaded per thread with the count
+        uint2 v[kCL];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = __ldcg(cand + min(rt + k * NT, P.ns - 1));
+        for (int k = 0; k < kCL; ++k) v[k] = __ldcg(cand + min(rt + k * NT, P.ns - 1));
         // with them, the sequence's histogram of key bits [19:10] over digit D1
         const uint4* gh2 = reinterpret_cast<const uint4*>(P.ghist2 + (int64_t)b * 1024);
         constexpr int kH2 = (256 + NT - 1) / NT;
@@ -888,18 +889,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint2* sc = reinterpret_cast<uint2*>(ring + kCandOff);
         if (in_smem) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < kCL; ++k) {
                 const int i = rt + k * NT;
                 if (i < C) sc[i] = v[k];
             }
-            for (int i0 = 8 * NT; i0 < C; i0 += 8 * NT) {  // 8 loads in flight per thread
+            for (int i0 = kCL * NT; i0 < C; i0 += kCL * NT) {  // kCL loads in flight per thread
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < kCL; ++k) {
                     const int i = i0 + rt + k * NT;
                     if (i < C) v[k] = __ldcg(cand + i);
                 }
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < kCL; ++k) {
                     const int i = i0 + rt + k * NT;
                     if (i < C) sc[i] = v[k];
                 }
@@ -1090,11 +1091,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = lo + tid; i < hi; i += kThreads) gh2[i] = 0u;
     }
     {
-        constexpr int kChunk = 16;  // partials loaded together
+        constexpr int kChunk = 24;  // partials loaded together (every CTA's at B = 8)
         const int c = tid & (kD - 1), sub = tid / kD;
         const int64_t jstride = (int64_t)P.H_q * (kD + 2);
         for (int h = j + sub * P.ncta; h < P.H_q; h += (kThreads / kD) * P.ncta) {
             const float* rec0 = P.part + ((int64_t)b * P.ncta * P.H_q + h) * (kD + 2);
+            // the gate logit and the linear branch's output load with the partials
+            const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + h]);
+            const float o_lin = __ldcg(P.olin + ((int64_t)b * P.H_q + h) * kD + c);
             float Mx = -INFINITY, Lsum = 0.0f, O = 0.0f;
 #pragma unroll 1
             for (int i0 = 0; i0 < P.ncta; i0 += kChunk) {
@@ -1127,8 +1131,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Mx = cm;
             }
             const float o_sp = Lsum > 0.0f ? O / Lsum : 0.0f;
-            const float x = __bfloat162float(P.gate[(int64_t)b * P.H_q + h]);
-            const float o_lin = __ldcg(P.olin + ((int64_t)b * P.H_q + h) * kD + c);
             const float gt = 1.0f / (1.0f + __expf(-x));
             P.o[((int64_t)b * P.H_q + h) * kD + c] = __float2bfloat16_rn(gt * o_lin + (1.0f - gt) * o_sp);
         }
