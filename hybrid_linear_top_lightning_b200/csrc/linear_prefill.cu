@@ -174,12 +174,12 @@ __global__ void __launch_bounds__(256) k_la_prefix(const LaParams P) {
         float run = P.S[e];
         float* U = P.U + bg * P.nch * per + el;
         int c = 0;
-        for (; c + 8 <= P.nch; c += 8) {
-            float u[8];
+        for (; c + 16 <= P.nch; c += 16) {  // 16 loads in flight per thread
+            float u[16];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) u[x] = U[(int64_t)(c + x) * per];
+            for (int x = 0; x < 16; ++x) u[x] = __ldcg(U + (int64_t)(c + x) * per);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
+            for (int x = 0; x < 16; ++x) {
                 U[(int64_t)(c + x) * per] = run;
                 run += u[x];
             }
@@ -383,18 +383,28 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         // S_{c-1} (fp32, row = key feature) into bf16 hi + lo, MN-major: row i of
         // value block jb at jb * 16384 + i * 128, chunk of 8 dims swizzled by i % 8
         const float* Sp = P.U + (((int64_t)b * P.H_kv + g) * P.nch + c) * kD * kD;
-        for (int rr = warp - 2; rr < kD; rr += 4) {
-            const float4 f = *reinterpret_cast<const float4*>(Sp + (int64_t)rr * kD + lane * 4);
-            const int j = lane * 4, jb = j >> 6, cc = (j & 63) >> 3;
-            const int off = jb * 16384 + rr * 128 + (((cc ^ (rr & 7)) << 4) | ((j & 7) << 1));
-            const __nv_bfloat162 h0 = __floats2bfloat162_rn(f.x, f.y), h1 = __floats2bfloat162_rn(f.z, f.w);
-            const float2 g0 = __bfloat1622float2(h0), g1 = __bfloat1622float2(h1);
-            const __nv_bfloat162 l0 = __floats2bfloat162_rn(f.x - g0.x, f.y - g0.y);
-            const __nv_bfloat162 l1 = __floats2bfloat162_rn(f.z - g1.x, f.w - g1.y);
-            *reinterpret_cast<uint2*>(shi + off) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
-            *reinterpret_cast<uint2*>(slo + off) =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
+        // eight rows in flight per warp (warp w % 4 takes rows w - 2, w + 2, ...)
+#pragma unroll 1
+        for (int r0 = warp - 2; r0 < kD; r0 += 4 * 8) {
+            float4 f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                f[u] = __ldcg(reinterpret_cast<const float4*>(Sp + (int64_t)(r0 + 4 * u) * kD + lane * 4));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int rr = r0 + 4 * u;
+                const int j = lane * 4, jb = j >> 6, cc = (j & 63) >> 3;
+                const int off = jb * 16384 + rr * 128 + (((cc ^ (rr & 7)) << 4) | ((j & 7) << 1));
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(f[u].x, f[u].y);
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(f[u].z, f[u].w);
+                const float2 g0 = __bfloat1622float2(h0), g1 = __bfloat1622float2(h1);
+                const __nv_bfloat162 l0 = __floats2bfloat162_rn(f[u].x - g0.x, f[u].y - g0.y);
+                const __nv_bfloat162 l1 = __floats2bfloat162_rn(f[u].z - g1.x, f[u].w - g1.y);
+                *reinterpret_cast<uint2*>(shi + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&h0),
+                                                                  *reinterpret_cast<const uint32_t*>(&h1));
+                *reinterpret_cast<uint2*>(slo + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&l0),
+                                                                  *reinterpret_cast<const uint32_t*>(&l1));
+            }
         }
         if (norm) zc[et] = P.Z[(((int64_t)b * P.H_kv + g) * P.nch + c) * kD + et];
         asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 2-5, unconditionally: z is in

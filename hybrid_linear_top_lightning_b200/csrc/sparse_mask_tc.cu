@@ -53,7 +53,8 @@ constexpr int kQT = 128;          // query rows per tile (MMA M)
 constexpr int kKT = 64;           // keys per tile
 constexpr int kD = 128;           // head dimension of this path
 constexpr int kStages = 4;        // K (and V) tiles in flight
-constexpr int kThreads = 320;     // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 softmax (two groups)
+constexpr int kThreads = 352;     // warp 0 TMA (Q, K), 1 MMA + TMEM, 2-9 softmax (two groups), 10 TMA (V)
+constexpr int kVWarp = 10;
 constexpr int kMaxTiles = 2048;   // key tiles one query tile may visit (keys <= 131072)
 constexpr uint32_t kTries = 1u << 22;
 constexpr float kLazy = 64.0f;    // move the softmax reference when a score exceeds it by more (log2)
@@ -226,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0 && n > 0) {
-            // ---- producer
+            // ---- producer of Q and the K tiles (V has its own warp, so a K
+            // tile's load never waits behind a V slot that a P.V still reads)
             bool ok = true;
             ptx::mbar_arrive_expect_tx(q_full, 2 * 16384);
             ptx::tma_load_3d(qs, &tmap_q, h * kD, q0, b, q_full);
@@ -234,31 +236,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i % kStages, use = i / kStages;
-                const int key0 = list[i] * kKT;
                 if (use > 0) ok = wait_bar(&k_empty[s], (use - 1) & 1);
                 if (!ok) break;
                 ptx::mbar_arrive_expect_tx(&k_full[s], 16384);
-                ptx::tma_load_3d(ks + s * 16384, &tmap_k, g * kD, key0, b, &k_full[s]);
-                ptx::tma_load_3d(ks + s * 16384 + 8192, &tmap_k, g * kD + 64, key0, b, &k_full[s]);
-                if (use > 0) ok = wait_bar(&v_empty[s], (use - 1) & 1);
-                if (!ok) {
-                    // the K copies just issued land before the CTA may leave
-                    wait_bar(&k_full[s], use & 1);
-                    break;
-                }
-                ptx::mbar_arrive_expect_tx(&v_full[s], 16384);
-                ptx::tma_load_3d(vs + s * 16384, &tmap_v, g * kD, key0, b, &v_full[s]);
-                ptx::tma_load_3d(vs + s * 16384 + 8192, &tmap_v, g * kD + 64, key0, b, &v_full[s]);
+                ptx::tma_load_3d(ks + s * 16384, &tmap_k, g * kD, list[i] * kKT, b, &k_full[s]);
+                ptx::tma_load_3d(ks + s * 16384 + 8192, &tmap_k, g * kD + 64, list[i] * kKT, b, &k_full[s]);
                 issued = i + 1;
             }
             if (!ok) {
                 misc[2] = 1u;
                 record_error(P.status, kDevTimeout);
                 // copies still in flight land before the shared memory is released
-                for (int i = max(0, issued - kStages); i < issued; ++i) {
+                for (int i = max(0, issued - kStages); i < issued; ++i)
                     ptx::mbar_wait_bounded(&k_full[i % kStages], (i / kStages) & 1, 1u << 16);
+            }
+        }
+    } else if (warp == kVWarp) {
+        if (lane == 0 && n > 0) {
+            // ---- producer of the V tiles
+            bool ok = true;
+            int issued = 0;
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i % kStages, use = i / kStages;
+                if (use > 0) ok = wait_bar(&v_empty[s], (use - 1) & 1);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(&v_full[s], 16384);
+                ptx::tma_load_3d(vs + s * 16384, &tmap_v, g * kD, list[i] * kKT, b, &v_full[s]);
+                ptx::tma_load_3d(vs + s * 16384 + 8192, &tmap_v, g * kD + 64, list[i] * kKT, b, &v_full[s]);
+                issued = i + 1;
+            }
+            if (!ok) {
+                misc[2] = 1u;
+                record_error(P.status, kDevTimeout);
+                for (int i = max(0, issued - kStages); i < issued; ++i)
                     ptx::mbar_wait_bounded(&v_full[i % kStages], (i / kStages) & 1, 1u << 16);
-                }
             }
         }
     } else if (warp == 1) {
@@ -286,11 +297,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::umma_commit(&k_empty[s]);
                 ptx::umma_commit(&s_full[sb]);
             };
-            // the score products run two tiles ahead of the P.V products, so a
+            // the score products run three tiles ahead of the P.V products, so a
             // softmax group finds its next tile's scores ready when it finishes one
             int next_s = 0;
             for (int i = 0; i < n && ok; ++i) {
-                while (ok && next_s < n && next_s <= i + 2) issue_s(next_s++);
+                // (score buffer (i + 3) % 4 was released by tile i - 1's group,
+                // whose P tile this thread has already seen)
+                while (ok && next_s < n && next_s <= i + 3) issue_s(next_s++);
                 const int s = i % kStages, grp = i & 1;
                 ok = ok && wait_bar(&p_full[grp], (i >> 1) & 1);
                 ok = ok && wait_bar(&v_full[s], (i / kStages) & 1);
