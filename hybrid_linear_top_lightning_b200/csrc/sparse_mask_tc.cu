@@ -13,21 +13,26 @@
 //  k_sel_mask:       one CTA per query row writes the row's selection as bits
 //                    (position s -> bit s) and marks, per 128-row query tile,
 //                    the 64-key tiles that any of its rows selects from.
-//  k_sparse_mask_tc: one CTA per (query tile, query head).  Warp 0 brings Q
-//                    (once) and the K and V tiles of the marked key tiles by
-//                    TMA (128-byte swizzle, 4-stage rings); warp 1 owns TMEM
-//                    and issues S = Q K^T (M = 128 queries, N = 64 keys,
-//                    K = 128 dims) into one of two TMEM score buffers and
-//                    O += P V (M = 128, N = 128 dims, K = 64 keys, V read
-//                    MN-major straight from its TMA tile) into the TMEM
-//                    output; warps 2-5 (one query row per thread, the row's
-//                    TMEM lane) read S, keep only the selected keys, update
-//                    the row's running reference and sum (the output is
-//                    rescaled in TMEM only when a selected score exceeds the
-//                    reference by more than 2^64, which leaves the result
-//                    exact), write P as bf16 into shared
-//                    memory in the MMA's swizzled layout, and at the end
-//                    normalise O and store it.
+//  k_sparse_mask_tc: one CTA per two (query tile, query head) units of one
+//                    KV head, normally two heads of the same query tile (the
+//                    same selections, the same K/V tiles), so every K/V tile
+//                    brought into shared memory feeds 256 query rows.  Warp 0
+//                    brings both units' Q tiles (once) and the K tiles, warp 10
+//                    the V tiles, of the key tiles either unit marks (TMA,
+//                    128-byte swizzle, 4-stage rings); warp 1 owns TMEM and
+//                    issues, per key tile and unit in turn, S_u = Q_u K^T
+//                    (M = 128 queries, N = 64 keys, K = 128 dims) into one of
+//                    the unit's two TMEM score buffers and O_u += P_u V
+//                    (M = 128, N = 128 dims, K = 64 keys; P read from TMEM, V
+//                    MN-major straight from its TMA tile) into the unit's TMEM
+//                    output; warps 2-5 (unit 0) and 6-9 (unit 1), one query row
+//                    per thread (the row's TMEM lane), read S, keep only the
+//                    selected keys, update the row's running reference and sum
+//                    (the output is rescaled in TMEM only when a selected score
+//                    exceeds the reference by more than 2^64, which leaves the
+//                    result exact), write P as bf16 over the first half of the
+//                    scores it came from, and at the end normalise O and store
+//                    it.
 //
 // Every wait is bounded; one that gives up records LISA_ERR_TIMEOUT, and the
 // kernel waits (bounded) for its own copies and MMAs in flight, releases its
@@ -53,14 +58,13 @@ constexpr int kQT = 128;          // query rows per tile (MMA M)
 constexpr int kKT = 64;           // keys per tile
 constexpr int kD = 128;           // head dimension of this path
 constexpr int kStages = 4;        // K (and V) tiles in flight
-constexpr int kThreads = 352;     // warp 0 TMA (Q, K), 1 MMA + TMEM, 2-9 softmax (two groups), 10 TMA (V)
+constexpr int kThreads = 352;     // warp 0 TMA (Q, K), 1 MMA + TMEM, 2-9 softmax (one group per unit), 10 TMA (V)
 constexpr int kVWarp = 10;
-constexpr int kMaxTiles = 2048;   // key tiles one query tile may visit (keys <= 131072)
-constexpr uint32_t kTries = 1u << 22;
+constexpr int kMaxTiles = 2048;   // key tiles of a context this path takes (keys <= 131072)
+constexpr uint32_t kTries = 1u << 22;  // polls of a wait (each 64 ns or more in the MMA issuer)
 constexpr float kLazy = 64.0f;    // move the softmax reference when a score exceeds it by more (log2)
-constexpr uint32_t kTmemCols = 512;  // 4 score buffers at columns 0-255, the groups' outputs at 256, 384
-constexpr int kSBuf = 4;             // score buffers: tile i uses i % 4 (group i % 2 owns two)
-constexpr uint32_t kOCol = kSBuf * kKT;
+constexpr uint32_t kTmemCols = 512;  // score buffers (2 per unit) at columns 0-255, the units' outputs at 256, 384
+constexpr uint32_t kOCol = 4 * kKT;
 
 struct MaskParams {
     int T, n_past, M, Lw, nqt, nkw;
@@ -110,7 +114,7 @@ __global__ void __launch_bounds__(256) k_sel_mask(const MaskParams P) {
 }
 
 struct AttnParams {
-    int B, T, H_q, group, nqt, Lw, nkw;
+    int B, T, H_q, H_kv, group, nqt, Lw, nkw, slots;
     float scale_log2;
     const uint32_t* mask;
     const uint32_t* occ;
@@ -119,15 +123,12 @@ struct AttnParams {
 };
 
 struct Smem {
-    static constexpr int q = 0;                                  // 2 boxes of 64 dims x 128 rows
-    static constexpr int k = q + 2 * 16384;                      // kStages x (2 x 64 dims x 64 keys)
+    static constexpr int q = 0;                                  // 2 units x 2 boxes of 64 dims x 128 rows
+    static constexpr int k = q + 2 * 2 * 16384;                  // kStages x (2 x 64 dims x 64 keys)
     static constexpr int v = k + kStages * 16384;                // the same for V
-    static constexpr int p = v + kStages * 16384;                // 2 groups x 128 rows x 64 keys bf16
-    static constexpr int list = p + 2 * 16384;                   // int[kMaxTiles]
-    static constexpr int bars = list + kMaxTiles * 4;            // mbarriers
+    static constexpr int bars = v + kStages * 16384;             // mbarriers
     static constexpr int misc = bars + 32 * 8;                   // tmem base, tile count, fail
-    static constexpr int xch = misc + 64;                        // group 1's max and sum per row
-    static constexpr int total = xch + 2 * kQT * 4 + 1024;       // + base alignment slack
+    static constexpr int total = misc + 64 + 1024;               // + base alignment slack
 };
 static_assert(Smem::total <= 227 * 1024, "shared memory per CTA");
 
@@ -135,40 +136,92 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
     return ptx::mbar_wait_bounded(bar, parity, kTries);
 }
 
+// Walks the key tiles that either unit of the CTA visits (the OR of the two
+// query tiles' marks), in ascending order.
+struct TileCursor {
+    const uint32_t* a;
+    const uint32_t* b;
+    int nkw, w;
+    uint32_t bits;
+    __device__ TileCursor(const uint32_t* a_, const uint32_t* b_, int nkw_)
+        : a(a_), b(b_), nkw(nkw_), w(-1), bits(0u) {}
+    __device__ __forceinline__ int next() {
+        while (bits == 0u && w + 1 < nkw) {
+            ++w;
+            bits = __ldg(a + w) | __ldg(b + w);
+        }
+        if (bits == 0u) return 0;  // past the last mark (callers stop at the count)
+        const int t = w * 32 + __ffs(bits) - 1;
+        bits &= bits - 1u;
+        return t;
+    }
+};
+
+// The two (query tile, query head) units of a CTA.  Per (sequence, KV head g,
+// query tile) there are `slots` CTAs: slot j < group/2 takes heads 2j and
+// 2j+1 of the group on that query tile; with an odd group the last slot
+// takes the group's last head on two neighbouring query tiles (qt, qt-1),
+// counted down from the last tile, so that slot is empty on every other
+// tile; a lone first tile pairs with itself and its second copy stores
+// nothing.
+struct Units {
+    int b, g, qt[2], h[2];
+    bool live, dup;
+};
+
+__device__ __forceinline__ Units cta_units(const AttnParams& P) {
+    Units u;
+    const int slot = blockIdx.x % P.slots;
+    int rest = blockIdx.x / P.slots;
+    u.g = rest % P.H_kv;
+    rest /= P.H_kv;
+    u.b = rest % P.B;
+    const int qt = P.nqt - 1 - rest / P.B;  // longest query tiles first
+    const int npair = P.group / 2;
+    u.live = true;
+    u.dup = false;
+    if (slot < npair) {
+        u.qt[0] = u.qt[1] = qt;
+        u.h[0] = u.g * P.group + 2 * slot;
+        u.h[1] = u.h[0] + 1;
+    } else {
+        u.h[0] = u.h[1] = u.g * P.group + P.group - 1;
+        u.live = ((P.nqt - 1 - qt) & 1) == 0;
+        u.qt[0] = qt;
+        u.qt[1] = qt > 0 ? qt - 1 : qt;
+        u.dup = qt == 0;
+    }
+    return u;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_sparse_mask_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const AttnParams P) {
+    const Units U = cta_units(P);
+    if (!U.live) return;  // (uniform over the CTA: nothing initialised yet)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* qs = base + Smem::q;
     uint8_t* ks = base + Smem::k;
     uint8_t* vs = base + Smem::v;
-    uint8_t* ps = base + Smem::p;
-    int* list = reinterpret_cast<int*>(base + Smem::list);
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + Smem::bars);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
     uint64_t* k_empty = k_full + kStages;
     uint64_t* v_full = k_empty + kStages;
     uint64_t* v_empty = v_full + kStages;
-    uint64_t* s_full = v_empty + kStages;   // [4] score buffer i % 4 written
-    uint64_t* s_empty = s_full + kSBuf;     // [4] and read by its softmax group
-    uint64_t* p_full = s_empty + kSBuf;     // [2] group's P tile written
-    uint64_t* pv_done = p_full + 2;         // [2] group's P.V product done
-    uint64_t* mma_all = pv_done + 2;        // every MMA this CTA issued has completed
-    float* xm = reinterpret_cast<float*>(base + Smem::xch);
-    float* xl = xm + kQT;
+    // per unit u and score buffer b (index u * 2 + b; key tile i uses buffer i % 2)
+    uint64_t* s_full = v_empty + kStages;   // scores written
+    uint64_t* p_full = s_full + 4;          // P written over the scores it came from
+    uint64_t* pv_done = p_full + 4;         // the P.V product that read it has completed
+    uint64_t* mma_all = pv_done + 4;        // every MMA this CTA issued has completed
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + Smem::misc);  // [0] tmem, [1] tiles, [2] fail
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // longest query tiles first; the heads of one query tile run side by side
-    // (they read the same K/V tiles)
-    const int per_qt = P.B * P.H_q;
-    const int qt = P.nqt - 1 - (int)(blockIdx.x / per_qt);
-    const int rem = blockIdx.x % per_qt;
-    const int b = rem / P.H_q, h = rem % P.H_q, g = h / P.group;
-    const int q0 = qt * kQT;
+    const int b = U.b, g = U.g;
+    const uint32_t* occ0 = P.occ + ((int64_t)b * P.nqt + U.qt[0]) * P.nkw;
+    const uint32_t* occ1 = P.occ + ((int64_t)b * P.nqt + U.qt[1]) * P.nkw;
 
     if (tid == 0) {
         ptx::mbar_init(q_full, 1);
@@ -178,11 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(&v_full[s], 1);
             ptx::mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < kSBuf; ++s) {
+        for (int s = 0; s < 4; ++s) {
             ptx::mbar_init(&s_full[s], 1);
-            ptx::mbar_init(&s_empty[s], 4);
-        }
-        for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&p_full[s], 4);
             ptx::mbar_init(&pv_done[s], 1);
         }
@@ -195,29 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_relinquish();
     }
     if (warp == 0) {
-        // the marked key tiles of this query tile, in ascending order
-        const uint32_t* oc = P.occ + ((int64_t)b * P.nqt + qt) * P.nkw;
-        int done = 0;
-        for (int w0 = 0; w0 < P.nkw; w0 += 32) {
-            const uint32_t word = (w0 + lane < P.nkw) ? __ldg(oc + w0 + lane) : 0u;
-            const int c = __popc(word);
-            int incl = c;
+        // how many key tiles the CTA visits
+        int c = 0;
+        for (int w = lane; w < P.nkw; w += 32) c += __popc(__ldg(occ0 + w) | __ldg(occ1 + w));
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            int at = done + incl - c;
-            uint32_t wv = word;
-            while (wv) {
-                const int bit = __ffs(wv) - 1;
-                wv &= wv - 1;
-                if (at < kMaxTiles) list[at] = (w0 + lane) * 32 + bit;
-                ++at;
-            }
-            done += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) misc[1] = (uint32_t)min(done, kMaxTiles);
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) misc[1] = (uint32_t)c;
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -227,20 +260,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0 && n > 0) {
-            // ---- producer of Q and the K tiles (V has its own warp, so a K
-            // tile's load never waits behind a V slot that a P.V still reads)
+            // ---- producer of both units' Q tiles and the K tiles (V has its
+            // own warp, so a K load never waits behind a V slot in use)
             bool ok = true;
-            ptx::mbar_arrive_expect_tx(q_full, 2 * 16384);
-            ptx::tma_load_3d(qs, &tmap_q, h * kD, q0, b, q_full);
-            ptx::tma_load_3d(qs + 16384, &tmap_q, h * kD + 64, q0, b, q_full);
+            ptx::mbar_arrive_expect_tx(q_full, 4 * 16384);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                ptx::tma_load_3d(qs + u * 32768, &tmap_q, U.h[u] * kD, U.qt[u] * kQT, b, q_full);
+                ptx::tma_load_3d(qs + u * 32768 + 16384, &tmap_q, U.h[u] * kD + 64, U.qt[u] * kQT, b, q_full);
+            }
+            TileCursor cur(occ0, occ1, P.nkw);
             int issued = 0;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i % kStages, use = i / kStages;
+                const int kt = cur.next();
                 if (use > 0) ok = wait_bar(&k_empty[s], (use - 1) & 1);
                 if (!ok) break;
                 ptx::mbar_arrive_expect_tx(&k_full[s], 16384);
-                ptx::tma_load_3d(ks + s * 16384, &tmap_k, g * kD, list[i] * kKT, b, &k_full[s]);
-                ptx::tma_load_3d(ks + s * 16384 + 8192, &tmap_k, g * kD + 64, list[i] * kKT, b, &k_full[s]);
+                ptx::tma_load_3d(ks + s * 16384, &tmap_k, g * kD, kt * kKT, b, &k_full[s]);
+                ptx::tma_load_3d(ks + s * 16384 + 8192, &tmap_k, g * kD + 64, kt * kKT, b, &k_full[s]);
                 issued = i + 1;
             }
             if (!ok) {
@@ -255,14 +293,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && n > 0) {
             // ---- producer of the V tiles
             bool ok = true;
+            TileCursor cur(occ0, occ1, P.nkw);
             int issued = 0;
             for (int i = 0; i < n && ok; ++i) {
                 const int s = i % kStages, use = i / kStages;
+                const int kt = cur.next();
                 if (use > 0) ok = wait_bar(&v_empty[s], (use - 1) & 1);
                 if (!ok) break;
                 ptx::mbar_arrive_expect_tx(&v_full[s], 16384);
-                ptx::tma_load_3d(vs + s * 16384, &tmap_v, g * kD, list[i] * kKT, b, &v_full[s]);
-                ptx::tma_load_3d(vs + s * 16384 + 8192, &tmap_v, g * kD + 64, list[i] * kKT, b, &v_full[s]);
+                ptx::tma_load_3d(vs + s * 16384, &tmap_v, g * kD, kt * kKT, b, &v_full[s]);
+                ptx::tma_load_3d(vs + s * 16384 + 8192, &tmap_v, g * kD + 64, kt * kKT, b, &v_full[s]);
                 issued = i + 1;
             }
             if (!ok) {
@@ -274,50 +314,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && n > 0) {
-            // ---- MMA issuer: S_i into score buffer i % 2; P_i V_i into the
-            // output of softmax group i % 2
+            // ---- MMA issuer.  Per unit u it issues, each as soon as its inputs
+            // are there (polling, so one unit never waits behind the other):
+            //   S_u(j) = Q_u K_j^T into score buffer j % 2, once K_j has landed and
+            //          the product that read P_u(j-2) from that buffer has completed;
+            //   O_u += P_u(i) V_i, with P_u(i) read from TMEM where the unit's
+            //          softmax wrote it over the first half of S_u(i), once P_u(i)
+            //          is written and V_i has landed.
+            // A K (V) slot is released when both units' products that read it
+            // are issued (the commit covers every earlier MMA).
             const uint32_t idesc_s = ptx::idesc_bf16_f32(kQT, kKT);
             const uint32_t idesc_pv = ptx::idesc_bf16_f32_bmn(kQT, kD);
-            const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs), qd1 = ptx::sdesc_kmajor_sw128(qs + 16384);
             bool ok = wait_bar(q_full, 0);
-            auto issue_s = [&](int i) {
-                const int s = i % kStages, sb = i % kSBuf;
-                ok = ok && wait_bar(&k_full[s], (i / kStages) & 1);
-                if (ok && i >= kSBuf) ok = wait_bar(&s_empty[sb], ((i / kSBuf) - 1) & 1);
-                if (!ok) return;
-                ptx::tc_fence_after();
-                const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
-                const uint64_t kd1 = ptx::sdesc_kmajor_sw128(ks + s * 16384 + 8192);
+            int ns0 = 0, ns1 = 0, np0 = 0, np1 = 0;  // next S / P.V tile per unit
+            uint32_t idle = 0;
+            while (ok && (np0 < n || np1 < n)) {
+                bool progress = false;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
-                    const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
-                    ptx::umma_f16(tmem + (uint32_t)(sb * kKT), a, bd, idesc_s, kk > 0);
+                for (int u = 0; u < 2; ++u) {
+                    int& ns = u ? ns1 : ns0;
+                    int& np = u ? np1 : np0;
+                    const int ns_other = u ? ns0 : ns1, np_other = u ? np0 : np1;
+                    const int j = ns;
+                    if (j < n && j <= np + 1) {
+                        const int s = j % kStages;
+                        bool ready = ptx::mbar_test(&k_full[s], (j / kStages) & 1);
+                        if (ready && j >= 2) ready = ptx::mbar_test(&pv_done[u * 2 + (j & 1)], ((j >> 1) - 1) & 1);
+                        if (ready) {
+                            ptx::tc_fence_after();
+                            const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
+                            const uint64_t kd1 = ptx::sdesc_kmajor_sw128(ks + s * 16384 + 8192);
+                            const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs + u * 32768);
+                            const uint64_t qd1 = ptx::sdesc_kmajor_sw128(qs + u * 32768 + 16384);
+#pragma unroll
+                            for (int kk = 0; kk < kD / 16; ++kk) {
+                                const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                                const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
+                                ptx::umma_f16(tmem + (uint32_t)((u * 2 + (j & 1)) * kKT), a, bd, idesc_s, kk > 0);
+                            }
+                            ptx::umma_commit(&s_full[u * 2 + (j & 1)]);
+                            if (ns_other > j) ptx::umma_commit(&k_empty[s]);
+                            ns = j + 1;
+                            progress = true;
+                        }
+                    }
+                    const int i = np;
+                    if (i < n && i < ns) {
+                        const int s = i % kStages;
+                        bool ready = ptx::mbar_test(&p_full[u * 2 + (i & 1)], (i >> 1) & 1);
+                        if (ready) ready = ptx::mbar_test(&v_full[s], (i / kStages) & 1);
+                        if (ready) {
+                            ptx::tc_fence_after();
+                            const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
+                            const uint32_t pt = tmem + (uint32_t)((u * 2 + (i & 1)) * kKT);
+#pragma unroll
+                            for (int kk = 0; kk < kKT / 16; ++kk)
+                                ptx::umma_f16_ts(tmem + kOCol + (uint32_t)(u * kD), pt + (uint32_t)(8 * kk),
+                                                 vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
+                                                 (i > 0 || kk > 0) ? 1u : 0u);
+                            ptx::umma_commit(&pv_done[u * 2 + (i & 1)]);
+                            if (np_other > i) ptx::umma_commit(&v_empty[s]);
+                            np = i + 1;
+                            progress = true;
+                        }
+                    }
                 }
-                ptx::umma_commit(&k_empty[s]);
-                ptx::umma_commit(&s_full[sb]);
-            };
-            // the score products run three tiles ahead of the P.V products, so a
-            // softmax group finds its next tile's scores ready when it finishes one
-            int next_s = 0;
-            for (int i = 0; i < n && ok; ++i) {
-                // (score buffer (i + 3) % 4 was released by tile i - 1's group,
-                // whose P tile this thread has already seen)
-                while (ok && next_s < n && next_s <= i + 3) issue_s(next_s++);
-                const int s = i % kStages, grp = i & 1;
-                ok = ok && wait_bar(&p_full[grp], (i >> 1) & 1);
-                ok = ok && wait_bar(&v_full[s], (i / kStages) & 1);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint64_t pd = ptx::sdesc_kmajor_sw128(ps + grp * 16384);
-                const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    ptx::umma_f16(tmem + kOCol + (uint32_t)(grp * kD), pd + 2 * kk,
-                                  vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
-                                  (i >= 2 || kk > 0) ? 1u : 0u);
-                ptx::umma_commit(&v_empty[s]);
-                ptx::umma_commit(&pv_done[grp]);
+                if (progress) {
+                    idle = 0;
+                } else {
+                    if (++idle > kTries) ok = false;
+                    __nanosleep(64);  // (leaves the issue slots to the softmax warps of this SMSP)
+                }
             }
             if (!ok) {
                 misc[2] = 1u;
@@ -328,47 +395,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_wait_bounded(mma_all, 0, kTries);
         }
     } else {
-        // ---- softmax: two groups of four warps take alternate key tiles
-        // (group grp: tiles grp, grp + 2, ...), each with its own running max
-        // and sum per row and its own output in TMEM; thread = query row
-        const int grp = (warp - 2) >> 2;
+        // ---- softmax: group u (four warps) takes unit u over every key
+        // tile, with the row's running reference and sum; thread = query row
+        const int u = (warp - 2) >> 2;
         const int lb = (warp & 3) * 32;
         const int r = lb + lane;
-        const int t = q0 + r;
+        const int t = (u == 0 ? U.qt[0] : U.qt[1]) * kQT + r;
+        const int h = u == 0 ? U.h[0] : U.h[1];
         const bool valid = t < P.T;
-        const uint32_t* mrow = P.mask + ((int64_t)b * P.T + (valid ? t : 0)) * P.Lw;
+        const uint2* mrow = reinterpret_cast<const uint2*>(P.mask + ((int64_t)b * P.T + (valid ? t : 0)) * P.Lw);
         const uint32_t t_row = tmem + ((uint32_t)lb << 16);
-        const uint32_t t_out = t_row + kOCol + (uint32_t)(grp * kD);  // and output
-        uint8_t* prow = ps + grp * 16384 + r * 128;
-        const int mine = grp < n ? (n - grp + 1) / 2 : 0;  // tiles of this group
+        const uint32_t t_out = t_row + kOCol + (uint32_t)(u * kD);
         float m_used = -INFINITY, l = 0.0f;
-        // the row's mask words of this group's next two tiles
+        // the row's mask words of the next two tiles
+        TileCursor cur(occ0, occ1, P.nkw);
         uint2 mk_a = make_uint2(0u, 0u), mk_b = make_uint2(0u, 0u);
-        if (valid && mine > 0) mk_a = __ldg(reinterpret_cast<const uint2*>(mrow) + list[grp]);
-        if (valid && mine > 1) mk_b = __ldg(reinterpret_cast<const uint2*>(mrow) + list[grp + 2]);
+        if (n > 0) {
+            const int t0 = cur.next();
+            if (valid) mk_a = __ldg(mrow + t0);
+        }
+        if (n > 1) {
+            const int t1 = cur.next();
+            if (valid) mk_b = __ldg(mrow + t1);
+        }
         bool ok = true;
-        for (int j = 0; j < mine; ++j) {
-            const int i = 2 * j + grp;
+        for (int i = 0; i < n; ++i) {
             const uint2 mk = mk_a;
             mk_a = mk_b;
-            if (valid && j + 2 < mine) mk_b = __ldg(reinterpret_cast<const uint2*>(mrow) + list[i + 4]);
-            const int sb = i % kSBuf;
-            const uint32_t t_s = t_row + (uint32_t)(sb * kKT);  // this tile's score buffer
+            if (i + 2 < n) {
+                const int tn = cur.next();
+                if (valid) mk_b = __ldg(mrow + tn);
+            }
+            const int sb = i & 1;
+            const uint32_t t_s = t_row + (uint32_t)((u * 2 + sb) * kKT);  // this tile's score buffer
             // (waits agree across the warp: the TMEM accesses that follow are collective)
-            if (!__all_sync(0xffffffffu, wait_bar(&s_full[sb], (i / kSBuf) & 1))) {
+            if (!__all_sync(0xffffffffu, wait_bar(&s_full[u * 2 + sb], (i >> 1) & 1))) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            // the tile's 64 scores, both loads in flight before the one wait;
-            // the score buffer is then free for the MMA to refill
+            // the tile's 64 scores, both loads in flight before the one wait
             uint32_t sr[64];
             ptx::tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(sr));
             ptx::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
             ptx::tmem_ld_wait();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&s_empty[sb]);
             // The reference m_used only has to keep every selected p = 2^(s - m_used)
             // far from overflow: the largest score of the whole tile (selected or
             // not, four chains) bounds the selected ones, so the masked maximum is
@@ -411,18 +481,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pk[k >> 1] = ptx::pack_bf16(p0, p1);
             }
             l = l * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
-            // this group's previous product has completed: its P tile is free
-            // and its output holds every product so far
-            if (j > 0 && !__all_sync(0xffffffffu, wait_bar(&pv_done[grp], (j - 1) & 1))) {
-                ok = false;
-                break;
-            }
-            // row r of P: 128 bytes, 16-byte chunk c at chunk c ^ (r % 8)
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            // P(i) as bf16 pairs over the first 32 columns of the score buffer
+            // (the A operand of the P.V product)
+            ptx::tmem_st32(t_s, *reinterpret_cast<const uint32_t(*)[32]>(pk));
             if (__any_sync(0xffffffffu, grow)) {
+                // the unit's previous product has completed: its output holds
+                // every product so far, and none is in flight until P(i) is out
+                if (i > 0 && !__all_sync(0xffffffffu, wait_bar(&pv_done[u * 2 + ((i - 1) & 1)], ((i - 1) >> 1) & 1))) {
+                    ok = false;
+                    break;
+                }
                 ptx::tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kD; c += 16) {
@@ -433,59 +501,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
                     ptx::tmem_st16(t_out + (uint32_t)c, ov);
                 }
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
             }
-            ptx::fence_proxy_async_shared();
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&p_full[grp]);
+            if (lane == 0) ptx::mbar_arrive(&p_full[u * 2 + sb]);
         }
         if (!ok) {
             misc[2] = 1u;
             if (lane == 0) record_error(P.status, kDevTimeout);
         }
-        // ---- epilogue: group 1 hands its (max, sum) over; group 0 merges the
-        // two outputs, divides by the sum and stores bf16
-        const bool have = __all_sync(0xffffffffu,
-                                     ok && (mine == 0 || wait_bar(&pv_done[grp], (mine - 1) & 1)));
-        if (grp == 1) {
-            xm[r] = have ? m_used : -INFINITY;
-            xl[r] = have ? l : 0.0f;
-        }
-        ptx::tc_fence_before();
-        asm volatile("bar.sync 1, 256;" ::: "memory");  // both groups, unconditionally
+        // ---- epilogue: divide the unit's output by the row's sum and store
+        // bf16 (zeros for a row that selected nothing)
+        const bool have = __all_sync(0xffffffffu, ok && n > 0 &&
+                                               wait_bar(&pv_done[u * 2 + ((n - 1) & 1)], ((n - 1) >> 1) & 1));
         ptx::tc_fence_after();
-        if (grp == 0) {
-            const float mb = xm[r], lb2 = xl[r];
-            const float ma = have ? m_used : -INFINITY;
-            const float mm = fmaxf(ma, mb);
-            const float ca = ma == -INFINITY ? 0.0f : exp2f(ma - mm);
-            const float cb = mb == -INFINITY ? 0.0f : exp2f(mb - mm);
-            const float lt = (have ? l : 0.0f) * ca + lb2 * cb;
-            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-            const float wa = ca * inv, wb = cb * inv;
-            bf16* orow = P.o + (((int64_t)b * P.T + (valid ? t : 0)) * P.H_q + h) * kD;
+        const float inv = (have && l > 0.0f) ? 1.0f / l : 0.0f;
+        bf16* orow = P.o + (((int64_t)b * P.T + (valid ? t : 0)) * P.H_q + h) * kD;
+        const bool store = valid && !(U.dup && u == 1);
 #pragma unroll 1
-            for (int c = 0; c < kD; c += 16) {
-                uint32_t oa[16], ob[16];
-                ptx::tmem_ld16(t_row + kOCol + (uint32_t)c, oa);
-                ptx::tmem_ld16(t_row + kOCol + kD + (uint32_t)c, ob);
+        for (int c = 0; c < kD; c += 16) {
+            uint32_t ov[16];
+            if (have) {
+                ptx::tmem_ld16(t_out + (uint32_t)c, ov);
                 ptx::tmem_ld_wait();
-                uint32_t pkd[8];
+            }
+            uint32_t pkd[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    // an output no product has written is never read (its weight is 0)
-                    const float a0 = wa != 0.0f ? __uint_as_float(oa[2 * e]) * wa : 0.0f;
-                    const float a1 = wa != 0.0f ? __uint_as_float(oa[2 * e + 1]) * wa : 0.0f;
-                    const float b0 = wb != 0.0f ? __uint_as_float(ob[2 * e]) * wb : 0.0f;
-                    const float b1 = wb != 0.0f ? __uint_as_float(ob[2 * e + 1]) * wb : 0.0f;
-                    pkd[e] = ptx::pack_bf16(a0 + b0, a1 + b1);
-                }
-                if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c);
-                    dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-                    dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
-                }
+            for (int e = 0; e < 8; ++e) {
+                // an output that no product has written is never read
+                const float a0 = inv != 0.0f ? __uint_as_float(ov[2 * e]) * inv : 0.0f;
+                const float a1 = inv != 0.0f ? __uint_as_float(ov[2 * e + 1]) * inv : 0.0f;
+                pkd[e] = ptx::pack_bf16(a0, a1);
+            }
+            if (store) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+                dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+                dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
             }
         }
     }
@@ -576,10 +628,13 @@ cudaError_t sparse_mask_attention(const Shape& s, const void* q, const void* k, 
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
     AttnParams ap;
-    ap.B = s.B; ap.T = s.T; ap.H_q = s.H_q; ap.group = s.group; ap.nqt = lay.nqt; ap.Lw = lay.Lw;
-    ap.nkw = lay.nkw; ap.scale_log2 = s.sm_scale * 1.4426950408889634f;
+    ap.B = s.B; ap.T = s.T; ap.H_q = s.H_q; ap.H_kv = s.H_kv; ap.group = s.group; ap.nqt = lay.nqt;
+    ap.Lw = lay.Lw; ap.nkw = lay.nkw; ap.slots = s.group / 2 + (s.group & 1);
+    ap.scale_log2 = s.sm_scale * 1.4426950408889634f;
     ap.mask = mask; ap.occ = occ; ap.o = static_cast<bf16*>(o); ap.status = static_cast<unsigned*>(ws);
-    k_sparse_mask_tc<<<s.B * lay.nqt * s.H_q, kThreads, Smem::total, st>>>(tq, tk, tv, ap);
+    const int64_t grid = (int64_t)s.B * lay.nqt * s.H_kv * ap.slots;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    k_sparse_mask_tc<<<(unsigned)grid, kThreads, Smem::total, st>>>(tq, tk, tv, ap);
     return cudaGetLastError();
 }
 

@@ -4,9 +4,12 @@ over 128-query x 64-key tiles on tcgen05 (LISA Sec. 3.2 Eq. 1, SA_M).
 
 The index rows here are seeded random sets, not top-M rows: any order, a
 count per row below the budget (zero included), rows past a partial last
-query tile, a call that continues after cached tokens, three head layouts,
-and logits large enough that the running maximum jumps by more than 2^8
-between key tiles (the output is then rescaled in TMEM).  Every row is
+query tile, a call that continues after cached tokens, head groups of 7, 6,
+8, 3 and 1 query heads per KV head (a CTA takes two heads of one query tile,
+or, for the odd head of a group, that head on two neighbouring query tiles,
+or on the first tile alone), and logits large enough that the running
+maximum jumps by more than 2^64 between key tiles (the output is then
+rescaled in TMEM).  Every row is
 compared with the oracle's sparse attention on the same index rows.
 Tolerance: max abs <= 2e-2 (bf16 outputs).
 """
@@ -69,7 +72,7 @@ def _case(wl, T, n_past, seed, q_scale=1.0, zero_every=0):
     return err
 
 
-@pytest.mark.parametrize("H_q,H_kv", [(28, 4), (12, 2), (8, 1)])
+@pytest.mark.parametrize("H_q,H_kv", [(28, 4), (12, 2), (8, 1), (6, 2), (4, 4)])
 def test_mask_path_random_rows_continued_call(H_q, H_kv):
     # 300 rows (a partial third query tile) after 150 cached tokens, 2 sequences
     wl = inputs.PREFILL_7B.with_(B=2, n=450, M=96, H_q=H_q, H_kv=H_kv)
