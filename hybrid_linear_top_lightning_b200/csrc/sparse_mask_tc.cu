@@ -19,8 +19,9 @@
 //                    brought into shared memory feeds 256 query rows.  Warp 0
 //                    brings both units' Q tiles (once) and the K tiles, warp 10
 //                    the V tiles, of the key tiles either unit marks (TMA,
-//                    128-byte swizzle, 4-stage rings); warp 1 owns TMEM and
-//                    issues, per key tile and unit in turn, S_u = Q_u K^T
+//                    128-byte swizzle, 4-stage rings); warp 1 owns TMEM, and
+//                    warps 1 and 11 each issue one unit's products, per key
+//                    tile S_u = Q_u K^T
 //                    (M = 128 queries, N = 64 keys, K = 128 dims) into one of
 //                    the unit's two TMEM score buffers and O_u += P_u V
 //                    (M = 128, N = 128 dims, K = 64 keys; P read from TMEM, V
@@ -58,10 +59,12 @@ constexpr int kQT = 128;          // query rows per tile (MMA M)
 constexpr int kKT = 64;           // keys per tile
 constexpr int kD = 128;           // head dimension of this path
 constexpr int kStages = 4;        // K (and V) tiles in flight
-constexpr int kThreads = 352;     // warp 0 TMA (Q, K), 1 MMA + TMEM, 2-9 softmax (one group per unit), 10 TMA (V)
+constexpr int kThreads = 384;     // warp 0 TMA (Q, K), 1 TMEM + MMA unit 0, 2-9 softmax (one group per unit),
+                                  // 10 TMA (V), 11 MMA unit 1
 constexpr int kVWarp = 10;
+constexpr int kMma1Warp = 11;
 constexpr int kMaxTiles = 2048;   // key tiles of a context this path takes (keys <= 131072)
-constexpr uint32_t kTries = 1u << 22;  // polls of a wait (each 64 ns or more in the MMA issuer)
+constexpr uint32_t kTries = 1u << 22;  // polls of a wait
 constexpr float kLazy = 64.0f;    // move the softmax reference when a score exceeds it by more (log2)
 constexpr uint32_t kTmemCols = 512;  // score buffers (2 per unit) at columns 0-255, the units' outputs at 256, 384
 constexpr uint32_t kOCol = 4 * kKT;
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* s_full = v_empty + kStages;   // scores written
     uint64_t* p_full = s_full + 4;          // P written over the scores it came from
     uint64_t* pv_done = p_full + 4;         // the P.V product that read it has completed
-    uint64_t* mma_all = pv_done + 4;        // every MMA this CTA issued has completed
+    uint64_t* mma_all = pv_done + 4;        // every MMA of both issuers has completed
     uint32_t* misc = reinterpret_cast<uint32_t*>(base + Smem::misc);  // [0] tmem, [1] tiles, [2] fail
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -227,16 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(q_full, 1);
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(&k_full[s], 1);
-            ptx::mbar_init(&k_empty[s], 1);
+            ptx::mbar_init(&k_empty[s], 2);  // one commit per unit's issuer
             ptx::mbar_init(&v_full[s], 1);
-            ptx::mbar_init(&v_empty[s], 1);
+            ptx::mbar_init(&v_empty[s], 2);
         }
         for (int s = 0; s < 4; ++s) {
             ptx::mbar_init(&s_full[s], 1);
             ptx::mbar_init(&p_full[s], 4);
             ptx::mbar_init(&pv_done[s], 1);
         }
-        ptx::mbar_init(mma_all, 1);
+        ptx::mbar_init(mma_all, 2);
         ptx::fence_mbar_init();
         misc[2] = 0u;
     }
@@ -312,79 +315,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_wait_bounded(&v_full[i % kStages], (i / kStages) & 1, 1u << 16);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kMma1Warp) {
         if (lane == 0 && n > 0) {
-            // ---- MMA issuer.  Per unit u it issues, each as soon as its inputs
-            // are there (polling, so one unit never waits behind the other):
-            //   S_u(j) = Q_u K_j^T into score buffer j % 2, once K_j has landed and
-            //          the product that read P_u(j-2) from that buffer has completed;
+            // ---- MMA issuer of unit u (one thread per unit: every tcgen05
+            // instruction costs its issuing thread tens of cycles, so one thread
+            // for both units would pace the tensor pipe).  Per key tile:
+            //   S_u(j) = Q_u K_j^T into score buffer j % 2, once K_j has landed
+            //          and the product that read P_u(j-2) from that buffer has
+            //          completed;
             //   O_u += P_u(i) V_i, with P_u(i) read from TMEM where the unit's
             //          softmax wrote it over the first half of S_u(i), once P_u(i)
             //          is written and V_i has landed.
-            // A K (V) slot is released when both units' products that read it
-            // are issued (the commit covers every earlier MMA).
+            // A K (V) slot is released when both issuers' products that read it
+            // have completed (one commit from each).
+            const int u = warp == 1 ? 0 : 1;
             const uint32_t idesc_s = ptx::idesc_bf16_f32(kQT, kKT);
             const uint32_t idesc_pv = ptx::idesc_bf16_f32_bmn(kQT, kD);
+            const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs + u * 32768);
+            const uint64_t qd1 = ptx::sdesc_kmajor_sw128(qs + u * 32768 + 16384);
+            const uint32_t o_col = tmem + kOCol + (uint32_t)(u * kD);
             bool ok = wait_bar(q_full, 0);
-            int ns0 = 0, ns1 = 0, np0 = 0, np1 = 0;  // next S / P.V tile per unit
-            uint32_t idle = 0;
-            while (ok && (np0 < n || np1 < n)) {
-                bool progress = false;
+            auto issue_s = [&](int j) {
+                const int s = j % kStages, bi = u * 2 + (j & 1);
+                ok = ok && wait_bar(&k_full[s], (j / kStages) & 1);
+                if (j >= 2) ok = ok && wait_bar(&pv_done[bi], ((j >> 1) - 1) & 1);
+                if (!ok) return;
+                ptx::tc_fence_after();
+                const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
+                const uint64_t kd1 = ptx::sdesc_kmajor_sw128(ks + s * 16384 + 8192);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    int& ns = u ? ns1 : ns0;
-                    int& np = u ? np1 : np0;
-                    const int ns_other = u ? ns0 : ns1, np_other = u ? np0 : np1;
-                    const int j = ns;
-                    if (j < n && j <= np + 1) {
-                        const int s = j % kStages;
-                        bool ready = ptx::mbar_test(&k_full[s], (j / kStages) & 1);
-                        if (ready && j >= 2) ready = ptx::mbar_test(&pv_done[u * 2 + (j & 1)], ((j >> 1) - 1) & 1);
-                        if (ready) {
-                            ptx::tc_fence_after();
-                            const uint64_t kd0 = ptx::sdesc_kmajor_sw128(ks + s * 16384);
-                            const uint64_t kd1 = ptx::sdesc_kmajor_sw128(ks + s * 16384 + 8192);
-                            const uint64_t qd0 = ptx::sdesc_kmajor_sw128(qs + u * 32768);
-                            const uint64_t qd1 = ptx::sdesc_kmajor_sw128(qs + u * 32768 + 16384);
-#pragma unroll
-                            for (int kk = 0; kk < kD / 16; ++kk) {
-                                const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
-                                const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
-                                ptx::umma_f16(tmem + (uint32_t)((u * 2 + (j & 1)) * kKT), a, bd, idesc_s, kk > 0);
-                            }
-                            ptx::umma_commit(&s_full[u * 2 + (j & 1)]);
-                            if (ns_other > j) ptx::umma_commit(&k_empty[s]);
-                            ns = j + 1;
-                            progress = true;
-                        }
-                    }
-                    const int i = np;
-                    if (i < n && i < ns) {
-                        const int s = i % kStages;
-                        bool ready = ptx::mbar_test(&p_full[u * 2 + (i & 1)], (i >> 1) & 1);
-                        if (ready) ready = ptx::mbar_test(&v_full[s], (i / kStages) & 1);
-                        if (ready) {
-                            ptx::tc_fence_after();
-                            const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
-                            const uint32_t pt = tmem + (uint32_t)((u * 2 + (i & 1)) * kKT);
-#pragma unroll
-                            for (int kk = 0; kk < kKT / 16; ++kk)
-                                ptx::umma_f16_ts(tmem + kOCol + (uint32_t)(u * kD), pt + (uint32_t)(8 * kk),
-                                                 vd + (uint64_t)((2048 >> 4) * kk), idesc_pv,
-                                                 (i > 0 || kk > 0) ? 1u : 0u);
-                            ptx::umma_commit(&pv_done[u * 2 + (i & 1)]);
-                            if (np_other > i) ptx::umma_commit(&v_empty[s]);
-                            np = i + 1;
-                            progress = true;
-                        }
-                    }
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+                    const uint64_t bd = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
+                    ptx::umma_f16(tmem + (uint32_t)(bi * kKT), a, bd, idesc_s, kk > 0);
                 }
-                if (progress) {
-                    idle = 0;
-                } else {
-                    if (++idle > kTries) ok = false;
-                    __nanosleep(64);  // (leaves the issue slots to the softmax warps of this SMSP)
-                }
+                ptx::umma_commit(&s_full[bi]);
+                ptx::umma_commit(&k_empty[s]);
+            };
+            issue_s(0);
+            if (n > 1) issue_s(1);
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i % kStages, bi = u * 2 + (i & 1);
+                ok = ok && wait_bar(&v_full[s], (i / kStages) & 1);
+                ok = ok && wait_bar(&p_full[bi], (i >> 1) & 1);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint64_t vd = ptx::sdesc_mnmajor_sw128(vs + s * 16384, 8192, 1024);
+                const uint32_t pt = tmem + (uint32_t)(bi * kKT);
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    ptx::umma_f16_ts(o_col, pt + (uint32_t)(8 * kk), vd + (uint64_t)((2048 >> 4) * kk),
+                                     idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                ptx::umma_commit(&pv_done[bi]);
+                ptx::umma_commit(&v_empty[s]);
+                if (i + 2 < n) issue_s(i + 2);
             }
             if (!ok) {
                 misc[2] = 1u;
@@ -446,7 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // first selected keys, or when it exceeds the reference by 2^kLazy.
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int k = 0; k < 64; ++k) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sr[k]));
+            for (int k = 0; k < 64; k += 2)
+                m4[(k >> 1) & 3] = ptx::max3(m4[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
             const bool any_sel = (mk.x | mk.y) != 0u;
             if (any_sel && (m_used == -INFINITY || mx > m_used + kLazy)) {
@@ -469,18 +454,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = grow ? exp2f(m_used - mx) : 1.0f;
             if (first || grow) m_used = mx;
             // probabilities of the selected keys (bf16 pairs), zero elsewhere
+            // (exponent arguments and partial sums two at a time: paired fp32 ops)
             uint32_t pk[32];
-            float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(-m_used, -m_used);
+            float2 l2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
             for (int k = 0; k < 64; k += 2) {
                 const uint32_t w = k < 32 ? mk.x : mk.y;
                 const bool s0 = (w & (1u << (k & 31))) != 0u, s1 = (w & (1u << ((k + 1) & 31))) != 0u;
-                const float p0 = s0 ? ptx::ex2(fmaf(__uint_as_float(sr[k]), P.scale_log2, -m_used)) : 0.0f;
-                const float p1 = s1 ? ptx::ex2(fmaf(__uint_as_float(sr[k + 1]), P.scale_log2, -m_used)) : 0.0f;
-                l4[(k >> 1) & 3] += p0 + p1;
+                const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sc2, nm2);
+                const float p0 = s0 ? ptx::ex2(x.x) : 0.0f;
+                const float p1 = s1 ? ptx::ex2(x.y) : 0.0f;
+                l2[(k >> 1) & 1] = ptx::add2(l2[(k >> 1) & 1], make_float2(p0, p1));
                 pk[k >> 1] = ptx::pack_bf16(p0, p1);
             }
-            l = l * alpha + ((l4[0] + l4[1]) + (l4[2] + l4[3]));
+            l = l * alpha + ((l2[0].x + l2[1].x) + (l2[0].y + l2[1].y));
             // P(i) as bf16 pairs over the first 32 columns of the score buffer
             // (the A operand of the P.V product)
             ptx::tmem_st32(t_s, *reinterpret_cast<const uint32_t(*)[32]>(pk));
