@@ -844,9 +844,13 @@ def prefill_work(wl) -> dict:
     # Q K^T (C x C x d, causal half) and P V (C x C x d, causal half)
     lin = nc * (wl.H_kv * 2 * wl.d * wl.d * C
                 + wl.H_q * (2 * C * wl.d * wl.d + 2 * 2 * (C * (C + 1) // 2) * wl.d))
-    gather = visits * wl.H_kv * wl.d * 2 * 2
+    # the masked tensor-core attention runs 128-query x 64-key tiles: every
+    # 64-key tile of a 128-row query tile's causal range that one of its rows
+    # selects from (all of them for these selections) costs the full tile
+    tiles = sum((min((qt + 1) * 128, n) + 63) // 64 for qt in range((n + 127) // 128))
+    sparse_tiles = tiles * wl.H_q * 128 * 64 * wl.d * 2 * 2
     return dict(pairs=pairs * wl.B, visits=visits * wl.B, indexer=indexer * wl.B,
-                sparse=sparse * wl.B, linear=lin * wl.B, gather_bytes=gather * wl.B,
+                sparse=sparse * wl.B, linear=lin * wl.B, sparse_tiles=sparse_tiles * wl.B,
                 total=(indexer + sparse + lin) * wl.B)
 
 
@@ -911,6 +915,8 @@ def run_prefill(args, wl, device):
     idx_tf = work["indexer"] / (times["topm"] / 1e3) / 1e12
     lin_tf = work["linear"] / (times["linear"] / 1e3) / 1e12
     lin_e_tf = work["linear"] / (times["linear_elu1"] / 1e3) / 1e12
+    sp_tf = work["sparse"] / (times["sparse_attn"] / 1e3) / 1e12
+    sp_tile_tf = work["sparse_tiles"] / (times["sparse_attn"] / 1e3) / 1e12
     return {
         "workload": wl.name, "B": B, "n": n, "M": wl.M, "H_q": wl.H_q, "H_kv": wl.H_kv,
         "value": B * n / whole_s, "unit": "tok/s", "ms": times["whole"], "steps": steps,
@@ -920,7 +926,8 @@ def run_prefill(args, wl, device):
         "gpu_launches_per_prefill": 7,
         "l2": "256 MB buffer written before every timed call",
         "work": {"indexer_gflop": work["indexer"] / 1e9, "sparse_gflop": work["sparse"] / 1e9,
-                 "linear_gflop": work["linear"] / 1e9, "gather_gb": work["gather_bytes"] / 1e9},
+                 "sparse_tile_gflop": work["sparse_tiles"] / 1e9,
+                 "linear_gflop": work["linear"] / 1e9},
         "roofline": {
             "bound": "tensor", "unit": "TFLOP/s", "peak": tc_burst, "peak_kind": peak_kind,
             "achieved": work["total"] / whole_s / 1e12,
@@ -928,7 +935,11 @@ def run_prefill(args, wl, device):
             "indexer_tflops_incl_select": idx_tf, "indexer_frac_incl_select": idx_tf / tc_burst,
             "linear_tflops": lin_tf, "linear_frac": lin_tf / tc_burst,
             "linear_elu1_tflops": lin_e_tf, "linear_elu1_frac": lin_e_tf / tc_burst,
-            "sparse_gather_gbs": work["gather_bytes"] / (times["sparse_attn"] / 1e3) / 1e9,
+            "sparse_attn_tflops_selected": sp_tf, "sparse_attn_frac_selected": sp_tf / tc_burst,
+            "sparse_attn_tflops_tiles": sp_tile_tf, "sparse_attn_frac_tiles": sp_tile_tf / tc_burst,
+            "sparse_attn_note": "selected = the selected (query, key) pairs' products; tiles = "
+                                "the products the tensor cores run over whole 128x64 tiles "
+                                "(unselected keys are dropped in the softmax)",
             "traffic": None},
     }
 
