@@ -65,7 +65,7 @@ constexpr int kVWarp = 10;
 constexpr int kMma1Warp = 11;
 constexpr int kMaxTiles = 2048;   // key tiles of a context this path takes (keys <= 131072)
 constexpr uint32_t kTries = 1u << 22;  // polls of a wait
-constexpr float kLazy = 64.0f;    // move the softmax reference when a score exceeds it by more (log2)
+constexpr float kLazyP = 1.8446744e19f;  // 2^64: a tile sum above this moves the softmax reference
 constexpr uint32_t kTmemCols = 512;  // score buffers (2 per unit) at columns 0-255, the units' outputs at 256, 384
 constexpr uint32_t kOCol = 4 * kKT;
 
@@ -424,51 +424,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
             ptx::tmem_ld_wait();
             // The reference m_used only has to keep every selected p = 2^(s - m_used)
-            // far from overflow: the largest score of the whole tile (selected or
-            // not, four chains) bounds the selected ones, so the masked maximum is
-            // taken only when that bound could move the reference: for the row's
-            // first selected keys, or when it exceeds the reference by 2^kLazy.
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int k = 0; k < 64; k += 2)
-                m4[(k >> 1) & 3] = ptx::max3(m4[(k >> 1) & 3], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
-            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
-            const bool any_sel = (mk.x | mk.y) != 0u;
-            if (any_sel && (m_used == -INFINITY || mx > m_used + kLazy)) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const uint32_t w = k < 32 ? mk.x : mk.y;
-                    if (w & (1u << (k & 31))) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sr[k]));
-                }
-                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
-            } else {
-                mx = -INFINITY;  // the reference stays
-            }
-            // the running max moves when a selected score exceeds it by more
-            // than 2^kLazy (the output and sum are rescaled by alpha then), or
-            // when the row meets its first selected key (its output is still zero)
-            const bool first = m_used == -INFINITY && mx != -INFINITY;
-            const bool grow = m_used != -INFINITY && mx > m_used + kLazy;
-            const float alpha = grow ? exp2f(m_used - mx) : 1.0f;
-            if (first || grow) m_used = mx;
-            // probabilities of the selected keys (bf16 pairs), zero elsewhere
-            // (exponent arguments and partial sums two at a time: paired fp32 ops)
+            // far from overflow.  So P is computed against the current reference
+            // and the tile's sum checked: only when it exceeds 2^64 (some
+            // selected score grew past the reference by about that much; +inf
+            // included) or the row meets its first selected keys is the masked
+            // maximum taken, the reference moved, and P computed again.  A row
+            // whose reference moves rescales its output and sum by alpha.
+            const uint32_t wlo = mk.x, whi = mk.y;
+            const float2 sc2 = make_float2(P.scale_log2, P.scale_log2);
             uint32_t pk[32];
-            const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(-m_used, -m_used);
-            float2 l2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float lt = 0.0f;
+            auto probs = [&](float ref) {
+                const float2 nm2 = make_float2(-ref, -ref);
+                float2 l2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-            for (int k = 0; k < 64; k += 2) {
-                const uint32_t w = k < 32 ? mk.x : mk.y;
-                const bool s0 = (w & (1u << (k & 31))) != 0u, s1 = (w & (1u << ((k + 1) & 31))) != 0u;
-                const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sc2, nm2);
-                const float p0 = s0 ? ptx::ex2(x.x) : 0.0f;
-                const float p1 = s1 ? ptx::ex2(x.y) : 0.0f;
-                l2[(k >> 1) & 1] = ptx::add2(l2[(k >> 1) & 1], make_float2(p0, p1));
-                pk[k >> 1] = ptx::pack_bf16(p0, p1);
+                for (int k = 0; k < 64; k += 2) {
+                    const uint32_t w = k < 32 ? wlo : whi;
+                    const bool s0 = (w & (1u << (k & 31))) != 0u, s1 = (w & (1u << ((k + 1) & 31))) != 0u;
+                    const float2 x = ptx::fma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), sc2, nm2);
+                    const float p0 = s0 ? ptx::ex2(x.x) : 0.0f;
+                    const float p1 = s1 ? ptx::ex2(x.y) : 0.0f;
+                    l2[(k >> 1) & 1] = ptx::add2(l2[(k >> 1) & 1], make_float2(p0, p1));
+                    pk[k >> 1] = ptx::pack_bf16(p0, p1);
+                }
+                lt = (l2[0].x + l2[1].x) + (l2[0].y + l2[1].y);
+            };
+            const bool any_sel = (wlo | whi) != 0u;
+            if (m_used != -INFINITY) probs(m_used);
+            // (the comparison is false for a NaN sum: NaN scores stay NaN)
+            const bool redo = any_sel && (m_used == -INFINITY || lt > kLazyP);
+            float alpha = 1.0f;
+            bool grow = false;
+            if (__any_sync(0xffffffffu, redo)) {
+                if (redo) {
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int k = 0; k < 64; ++k) {
+                        const uint32_t w = k < 32 ? wlo : whi;
+                        if (w & (1u << (k & 31))) m4[k & 3] = fmaxf(m4[k & 3], __uint_as_float(sr[k]));
+                    }
+                    const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * P.scale_log2;
+                    grow = m_used != -INFINITY && mx > m_used;
+                    if (grow) alpha = exp2f(m_used - mx);
+                    if (m_used == -INFINITY || grow) m_used = mx;
+                }
+                // (every lane of the warp, with its own reference)
+                if (m_used != -INFINITY) probs(m_used);
             }
-            l = l * alpha + ((l2[0].x + l2[1].x) + (l2[0].y + l2[1].y));
+            if (m_used == -INFINITY) {  // nothing selected in the row so far
+                lt = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) pk[k] = 0u;
+            }
+            l = l * alpha + lt;
             // P(i) as bf16 pairs over the first 32 columns of the score buffer
             // (the A operand of the P.V product)
             ptx::tmem_st32(t_s, *reinterpret_cast<const uint32_t(*)[32]>(pk));
