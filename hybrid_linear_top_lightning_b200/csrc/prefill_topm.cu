@@ -8,9 +8,10 @@
 //   D[key, (query, head)] = K_I[key] . Q_I[query, head] is one tcgen05.mma
 //   chain of shape M=128 (keys) x N=32*H_I (query x head) x K=d_I=64, operands
 //   brought into shared memory by TMA (128-byte swizzle), accumulator in TMEM.
-//   Roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps 2-5
-//   read the accumulator (one TMEM lane = one key per thread) and reduce over
-//   the heads inside the thread: score = sum_h w[q,h] * ReLU(D[key, (q,h)]).
+//   Roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps 2-9
+//   read the accumulator (one TMEM lane = one key per thread; the two warps of
+//   a lane quarter take alternate 32-column chunks) and reduce over the heads
+//   inside the thread: score = sum_h w[q,h] * ReLU(D[key, (q,h)]).
 //   Stores are coalesced along keys.  Two CTAs share an SM, so one's epilogue
 //   overlaps the other's MMAs.
 // k_topm_rows_fast: one CTA per query row; the row comes into shared memory by
@@ -38,7 +39,8 @@ constexpr int kDI = 64;
 constexpr int kQT = 32;        // query rows per tile
 constexpr int kKT = 128;       // keys per tile (MMA M)
 constexpr int kKStages = 4;    // key tiles in flight
-constexpr int kScoreThreads = 192;
+constexpr int kScoreThreads = 192;      // the paper-form kernel: warp 0 TMA, 1 MMA, 2-5 epilogue
+constexpr int kScoreMainThreads = 320;  // k_index_scores_tc: warp 0 TMA, 1 MMA, 2-9 epilogue
 constexpr uint32_t kTries = 1u << 22;
 
 struct ScoreParams {
@@ -63,7 +65,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity) {
 }
 
 template <int HI>
-__global__ void __launch_bounds__(kScoreThreads, 2)
+__global__ void __launch_bounds__(kScoreMainThreads, 2)
     k_index_scores_tc(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const ScoreParams P) {
     extern __shared__ uint8_t smem_raw[];
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
             ptx::mbar_init(&k_empty[s], 1);
         }
         ptx::mbar_init(t_full, 1);
-        ptx::mbar_init(t_empty, 128);
+        ptx::mbar_init(t_empty, 256);
         ptx::fence_mbar_init();
         s_fail = 0;
     }
@@ -108,8 +110,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     }
     if (warp >= 2) {
         // head weights of this tile's queries
-        const int e = tid - 64;  // 0..127
-        for (int i = e; i < kQT * P.H_I; i += 128) {
+        const int e = tid - 64;  // 0..255
+        for (int i = e; i < kQT * P.H_I; i += 256) {
             const int ql = i / P.H_I, h = i % P.H_I;
             float v = 0.0f;
             if (ql < qrows) {
@@ -164,8 +166,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
             }
         }
     } else {
-        // ---- epilogue: thread = key (TMEM lane), columns = (query, head)
+        // ---- epilogue: thread = key (TMEM lane), columns = (query, head); the
+        // two warps of a lane quarter take alternate 32-column chunks
         const int lg = (warp & 3) * 32;
+        const int half = (warp - 2) >> 2;
         const int key_l = lg + lane;
         constexpr int qpc = 32 / HI;  // queries per 32-column chunk
         for (int kt = 0; kt < n_kt; ++kt) {
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
             ptx::tc_fence_after();
             const int key = kt * kKT + key_l;
 #pragma unroll 1
-            for (int c0 = 0; c0 < N; c0 += 32) {
+            for (int c0 = half * 32; c0 < N; c0 += 64) {
                 uint32_t r[32];
                 ptx::tmem_ld32(tmem + ((uint32_t)lg << 16) + (uint32_t)c0, r);
                 ptx::tmem_ld_wait();
@@ -505,10 +509,10 @@ cudaError_t fast_topm(const Shape& s, const void* q_I, const void* k_I, const fl
     const dim3 grid(s.B * P.nqt);
     if (heads) k_index_scores_heads_tc<<<grid, kScoreThreads, HeadsSmem::total, st>>>(tq, tk, P);
     else switch (s.H_I) {
-        case 1: k_index_scores_tc<1><<<grid, kScoreThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
-        case 2: k_index_scores_tc<2><<<grid, kScoreThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
-        case 4: k_index_scores_tc<4><<<grid, kScoreThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
-        default: k_index_scores_tc<8><<<grid, kScoreThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
+        case 1: k_index_scores_tc<1><<<grid, kScoreMainThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
+        case 2: k_index_scores_tc<2><<<grid, kScoreMainThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
+        case 4: k_index_scores_tc<4><<<grid, kScoreMainThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
+        default: k_index_scores_tc<8><<<grid, kScoreMainThreads, ScoreSmem::total, st>>>(tq, tk, P); break;
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
