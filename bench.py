@@ -736,6 +736,30 @@ def run_next_rows(args, wl, copies, D, stream):
                      "achieved": st_bytes / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                      "frac": st_bytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
                      "traffic": None}}
+    del states, g
+
+    # ---- one recurrent step of the linear branch alone (lisa_linear_decode) at
+    # the headline shape; 64 state sets in rotation (134 MB, larger than L2)
+    nsets = 64
+    sets = [dict(S=torch.randn(shape, device=stream.device) * 0.05,
+                 q=torch.randn(wl.B, 1, wl.H_q, wl.d, device=stream.device).to(torch.bfloat16),
+                 k=torch.randn(wl.B, 1, wl.H_kv, wl.d, device=stream.device).to(torch.bfloat16),
+                 v=torch.randn(wl.B, 1, wl.H_kv, wl.d, device=stream.device).to(torch.bfloat16),
+                 o=torch.empty(wl.B, 1, wl.H_q, wl.d, device=stream.device, dtype=torch.bfloat16))
+            for _ in range(nsets)]
+    ms = graph_timed([lambda c=c: lisa.lisa_linear_decode(D, c["q"], c["k"], c["v"], c["S"], None, c["o"])
+                      for c in sets], args.steps, args.warmup)
+    ld_bytes = 2 * wl.B * wl.H_kv * wl.d * wl.d * 4 + 2 * wl.B * (2 * wl.H_q + 2 * wl.H_kv) * wl.d
+    out["linear_decode"] = {
+        "what": "one recurrent step of the linear branch (lisa_linear_decode, identity map): "
+                "S += phi(k)^T v, o = phi(q) S over B x H_kv states of d x d fp32",
+        "us_per_call": ms * 1e3,
+        "l2": f"{nsets} state sets in rotation ({nsets * wl.B * wl.H_kv * wl.d * wl.d * 4 / 1e6:.0f} MB, "
+              "larger than L2); a CUDA graph of one call per set replayed",
+        "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": ld_bytes,
+                     "achieved": ld_bytes / (ms / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": ld_bytes / (ms / 1e3) / 1e9 / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": None}}
     return out
 
 
@@ -991,6 +1015,38 @@ def oracle_decode_sample(wl, seqs: int, budget_s: float):
                         f"thread(s)")
 
 
+def oracle_prefill_sample(wl, stride: int, budget_s: float):
+    """Time the oracle's whole module on every `stride`-th query row of one
+    causal prefill of the workload (each sampled row: the indexer over all its
+    causal keys, a full sort, sparse attention and the gate; the linear
+    recurrence runs over every token), repeated until about `budget_s` seconds
+    have passed.  Returns (sampled rows per second, threads, note)."""
+    from hybrid_linear_top_lightning_b200 import inputs
+    from oracle import ref
+
+    gen = inputs.Generator(wl)
+    n = wl.n
+    x = {k: gen.batch(k, 0, n) for k in ("q", "k", "v", "q_I", "k_I", "w", "gate")}
+    D = ref.Dims(B=wl.B, T=n, n_past=0, N_max=n, H_q=wl.H_q, H_kv=wl.H_kv, d=wl.d, H_I=wl.H_I,
+                 H_Ik=wl.H_Ik, d_I=wl.d_I, M=wl.M)
+    rows = np.arange(stride - 1, n, stride, dtype=np.int32)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        ref.forward(D, x["q"], x["k"], x["v"], x["q_I"], x["k_I"], x["w"], wl.H_I, x["q"], x["k"],
+                    x["v"], x["gate"], rows=rows)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    thr = ref.num_threads()
+    return reps * rows.size * wl.B / el, thr, (
+        f"{reps} oracle prefill pass(es) over every {stride}th query row ({rows.size} rows) of "
+        f"the {n}-token prefill (per sampled row: indexer over its causal keys, full sort, sparse "
+        f"attention, gate; the linear recurrence over all {n} tokens) in {el:.1f} s on {thr} "
+        f"thread(s)")
+
+
 def run_reference(args, wl):
     # rank 0 is the only worker of this arm, so it takes every core it may run
     # on (a multi-process launcher sets OMP_NUM_THREADS=1 for each rank)
@@ -1098,6 +1154,10 @@ def main():
                                     "kind": "oracle", "sample": note,
                                     "single_thread": {"value": tok_1, "unit": UNIT, "cores": 1,
                                                       "sample": note_1}}
+            if "prefill" in line:
+                pt, pc, pnote = oracle_prefill_sample(wl_p, stride=16, budget_s=args.cpu_seconds)
+                line["prefill"]["cpu_baseline"] = {"value": pt, "unit": "tok/s", "cores": pc,
+                                                   "kind": "oracle", "sample": pnote}
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

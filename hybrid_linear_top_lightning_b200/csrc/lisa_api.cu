@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include "lisa_internal.cuh"
+#include "linear_decode.cuh"
 #include "lisa_fast.cuh"
 
 namespace lisa {
@@ -237,6 +238,8 @@ lisa_status lisa_linear_decode(const lisa_dims* dims, const void* q_L, const voi
     if (s.B == 0) return LISA_OK;
     if (!q_L || !k_L || !v_L || !S || !o_lin) return LISA_ERR_INVALID_ARG;
     if (s.phi == LISA_PHI_ELU1_NORM && !z) return LISA_ERR_INVALID_ARG;
+    if (fast_linear_decode_supported(s, q_L, k_L, v_L, S))
+        return cuda_status(fast_linear_decode(s, q_L, k_L, v_L, S, z, o_lin, (cudaStream_t)stream));
     return cuda_status(generic_linear(s, q_L, k_L, v_L, S, z, o_lin, false, (cudaStream_t)stream));
 }
 
