@@ -267,6 +267,26 @@ def _setup_decode(wl, device):
     return kc, vc, kIc, S, dev, host
 
 
+def _packed_inputs(tensors, alloc):
+    """One flat byte buffer from `alloc(nbytes)` holding every tensor of
+    `tensors` (same dtypes and shapes) at 256-byte-aligned offsets, so that a
+    step's inputs move in one copy.  Returns (flat buffer, dict of views)."""
+    import torch
+
+    lay, off = {}, 0
+    for k, t in tensors.items():
+        nb = t.numel() * t.element_size()
+        lay[k] = (off, nb)
+        off += (nb + 255) & ~255
+    flat = alloc(off)
+    views = {}
+    for k, t in tensors.items():
+        o, nb = lay[k]
+        views[k] = flat[o:o + nb].view(t.dtype).view(t.shape)
+        views[k].copy_(t)
+    return flat, views
+
+
 def run_gpu(args, wl, rank, world, device):
     import torch
     import torch.distributed as dist
@@ -275,6 +295,9 @@ def run_gpu(args, wl, rank, world, device):
 
     torch.manual_seed(0)
     kc0, vc0, kIc0, S0, dv0, host = _setup_decode(wl, device)
+    # a step's inputs live in one device buffer per state copy (views into it),
+    # so the end-to-end line moves them host to device in one copy
+    dev_alloc = lambda nb: torch.empty(nb, dtype=torch.uint8, device=device)  # noqa: E731
     B, n, p = wl.B, wl.n, wl.n - 1
     D = lisa.make_dims(B, 1, p, n, wl.H_q, wl.H_kv, wl.d, wl.H_I, wl.H_Ik, wl.d_I, wl.M)
     stream = torch.cuda.current_stream()
@@ -284,16 +307,16 @@ def run_gpu(args, wl, rank, world, device):
     copies = []
     for r in range(args.rotate):
         if r == 0:
-            kc, vc, kIc, S, dv = kc0, vc0, kIc0, S0, dv0
+            kc, vc, kIc, S = kc0, vc0, kIc0, S0
         else:
             kc, vc, kIc, S = kc0.clone(), vc0.clone(), kIc0.clone(), S0.clone()
-            dv = {k: v.clone() for k, v in dv0.items()}
+        flat, dv = _packed_inputs(dv0, dev_alloc)
         ws = lisa.workspace(D, lisa.LISA_OP_DECODE_STEP, device)
         o = torch.empty(B, 1, wl.H_q, wl.d, dtype=torch.bfloat16, device=device)
         a = lisa.decode_args(dv["q"], dv["k_new"], dv["v_new"], dv["q_I"], dv["k_I_new"],
                              dv["w"], wl.H_I, dv["q"], dv["k_new"], dv["v_new"], dv["gate"],
                              kc, vc, kIc, S, None, o)
-        copies.append(dict(dv=dv, ws=ws, o=o, a=a, S=S, kc=kc, vc=vc, kIc=kIc))
+        copies.append(dict(dv=dv, flat=flat, ws=ws, o=o, a=a, S=S, kc=kc, vc=vc, kIc=kIc))
 
     def step(i):
         c = copies[i % len(copies)]
@@ -353,22 +376,52 @@ def run_gpu(args, wl, rank, world, device):
     total_ms = max_over_ranks(statistics.median(blocks), device, world)
     del graph
 
-    # ---- end to end through the public API with host buffers
-    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(
-        torch.float32 if k == "w" else torch.bfloat16).pin_memory() for k, v in host.items()}
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs (packed in one pinned buffer laid out like the device
+    # one) host to device in one copy, runs lisa_decode_step and reads o back
+    pinned, _ = _packed_inputs(
+        {k: torch.from_numpy(np.ascontiguousarray(v)).to(torch.float32 if k == "w" else torch.bfloat16)
+         for k, v in host.items()},
+        lambda nb: torch.empty(nb, dtype=torch.uint8).pin_memory())
     o_host = torch.empty(copies[0]["o"].shape, dtype=torch.bfloat16).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in pinned.values())
+    h2d = pinned.numel()
     d2h = o_host.numel() * o_host.element_size()
 
-    def e2e_step(i):
-        c = copies[i % len(copies)]
-        for k, x in pinned.items():
-            c["dv"][k].copy_(x, non_blocking=True)
-        lisa.lisa_decode_step(D, c["a"], c["ws"], stream)
-        o_host.copy_(c["o"], non_blocking=True)
+    # The copies run on their own stream, pipelined as a serving loop would:
+    # step i+1's inputs go up while step i's kernel runs (into the state copy
+    # step i+1 uses, once the kernel that last read it is done), and o of step
+    # i comes down after that kernel.  Every step's bytes still cross inside the
+    # timed region, which ends when the last read-back has landed.
+    R = len(copies)
+    cstream = torch.cuda.Stream(device)
+    up = [torch.cuda.Event() for _ in range(R)]    # inputs of the copy's next step landed
+    done = [torch.cuda.Event() for _ in range(R)]  # the copy's last kernel finished
+    used = [False] * R
 
-    for i in range(max(1, args.warmup)):
-        e2e_step(i)
+    def upload(j):
+        slot = j % R
+        if used[slot]:
+            cstream.wait_event(done[slot])
+        with torch.cuda.stream(cstream):
+            copies[slot]["flat"].copy_(pinned, non_blocking=True)
+        up[slot].record(cstream)
+
+    def e2e_run(count):
+        upload(0)
+        for i in range(count):
+            slot = i % R
+            if i + 1 < count:
+                upload(i + 1)
+            stream.wait_event(up[slot])
+            lisa.lisa_decode_step(D, copies[slot]["a"], copies[slot]["ws"], stream)
+            done[slot].record(stream)
+            used[slot] = True
+            cstream.wait_event(done[slot])
+            with torch.cuda.stream(cstream):
+                o_host.copy_(copies[slot]["o"], non_blocking=True)
+        stream.wait_stream(cstream)
+
+    e2e_run(max(1, args.warmup))
     torch.cuda.synchronize()
     e_st = torch.cuda.Event(enable_timing=True)
     e_en = torch.cuda.Event(enable_timing=True)
@@ -376,8 +429,7 @@ def run_gpu(args, wl, rank, world, device):
         dist.barrier()
     torch.cuda.synchronize()
     e_st.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
+    e2e_run(args.steps)
     e_en.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_st.elapsed_time(e_en), device, world)
