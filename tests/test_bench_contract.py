@@ -48,3 +48,31 @@ def test_reference_arm_two_processes():
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
     _check_line(lines[0], 2)
+
+
+def test_packed_step_inputs_share_one_buffer():
+    """The end-to-end decode line moves a step's inputs in one copy: the views
+    that `_packed_inputs` returns hold the given values, sit at 256-byte-aligned
+    offsets of one flat buffer, and a copy of the whole buffer moves them all."""
+    import torch
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    g = torch.Generator().manual_seed(3)
+    src = {"q": torch.randn(8, 1, 28, 128, generator=g).to(torch.bfloat16),
+           "w": torch.rand(8, 1, 8, generator=g),
+           "gate": torch.randn(8, 1, 28, generator=g).to(torch.bfloat16)}
+    flat, views = bench._packed_inputs(src, lambda nb: torch.zeros(nb, dtype=torch.uint8))
+    base = flat.data_ptr()
+    for k, t in src.items():
+        v = views[k]
+        assert v.dtype == t.dtype and v.shape == t.shape and torch.equal(v, t)
+        assert (v.data_ptr() - base) % 256 == 0
+        assert base <= v.data_ptr() and v.data_ptr() + v.numel() * v.element_size() <= base + flat.numel()
+    flat2, views2 = bench._packed_inputs({k: torch.zeros_like(t) for k, t in src.items()},
+                                         lambda nb: torch.zeros(nb, dtype=torch.uint8))
+    assert flat2.numel() == flat.numel()
+    flat2.copy_(flat)
+    for k, t in src.items():
+        assert torch.equal(views2[k], t)
